@@ -1,0 +1,379 @@
+"""Benchmark of the DeepSeekMoE FP8 layer forward pass on B200.
+
+One step = the whole layer on one batch: route -> quant_1x128 -> permute ->
+grouped FP8 GEMM (256 routed experts top-8 + 1 shared, SwiGLU, requant,
+down) -> combine -> bias update. The workload is the full DeepSeek-V3 layer
+shape at prefill (T=8192 tokens, d=7168, 256 routed top-8 + 1 shared,
+I=2048), synthetic seeded inputs already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun), every rank runs its own replica on its own batch
+(weak scaling; the layer needs no exchange between replicas); the time is the
+max over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the plain float64 reference of the
+same layer) on the host cores, on a bounded sample of tokens per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DeepSeekMoE FP8 layer tokens/s + TFLOP/s, % FP8 tensor peak (1×B200)"
+CONFIG_NAME = "prefill"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def layer_flops(cfg, rows_routed=None):
+    """Algorithmic FLOPs of the expert GEMMs: 6*d*I per (token, expert) pair
+    (gate, up, down), routed pairs plus the shared expert on every token."""
+    P = cfg.T * cfg.K_r if rows_routed is None else rows_routed
+    return 6.0 * cfg.d * cfg.I * (P + cfg.T)
+
+
+def workload_desc(cfg):
+    return (f"DeepSeek-V3 MoE layer, prefill: T={cfg.T}, d={cfg.d}, {cfg.N_r} routed experts "
+            f"top-{cfg.K_r} + 1 shared, SwiGLU I={cfg.I}, E4M3 1x128/128x128 scales")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def _oracle_sample_setup(cfg, tokens, device="cuda"):
+    """Inputs of a small token sample and the oracle-quantised weights of the
+    experts it touches (untimed preparation)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+
+    import workloads
+    from oracle import moe as O
+    u = workloads.activations(cfg, device=device)[tokens].cpu().double().numpy()
+    e = workloads.centroids(cfg, device=device).cpu().double().numpy()
+    b = workloads.bias(cfg, device=device).cpu().double().numpy()
+    _, _, idx, _ = O.route(u, e, b, cfg.K_r)
+    slots = sorted(set(idx.reshape(-1).tolist()) | {cfg.N_r})
+    raw = {s: [x.cpu().double().numpy() for x in workloads.expert_weights(cfg, s, device=device)]
+           for s in slots}
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 8) as ex:
+        quant = dict(zip(slots, ex.map(lambda s: O.quantise_expert(*raw[s]), slots)))
+    return u, e, b, quant
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(cfg, n_tokens, steps, device="cuda"):
+    """Times the oracle forward on a sample of n_tokens tokens per step (the
+    same sample every step). Returns (tokens/s, seconds per step, sample desc)."""
+    import numpy as np
+
+    from oracle import moe as O
+    tokens = np.arange(n_tokens)
+    u, e, b, quant = _oracle_sample_setup(cfg, tokens, device)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
+    dt = (time.perf_counter() - t0) / steps
+    desc = (f"oracle forward (route, quant, permute, {len(quant)} expert FFNs incl. shared, "
+            f"combine, bias update) on tokens 0..{n_tokens - 1} of the {cfg.name} batch, "
+            f"weights pre-quantised by the oracle; {steps} steps")
+    return n_tokens / dt, dt, desc
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import workloads
+    from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workloads.CONFIGS[CONFIG_NAME]
+    peaks = _peaks()
+
+    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, device=dev)
+    for slot in range(cfg.N_r + 1):
+        w = workloads.expert_weights(cfg, slot, device=dev)
+        layer.load_expert(slot, *w)
+        del w
+    u = workloads.activations(cfg, device=dev)
+    e = workloads.centroids(cfg, device=dev)
+    b0 = workloads.bias(cfg, device=dev)
+    b = b0.clone()
+    stream = torch.cuda.current_stream(dev)
+    torch.cuda.synchronize(dev)
+
+    def step():
+        layer.forward(u, e, b, update_bias=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if B.moe_get_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        start.record(stream)
+        for i in range(K):
+            layer.route(u, e, b)
+            layer.quant(u)
+            layer.permute()
+            ev[i][0].record(stream)
+            layer.experts()
+            ev[i][1].record(stream)
+            layer.combine(u)
+            layer.bias_update(b)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(stop)
+    gemm_ms = [a.elapsed_time(z) for a, z in ev]
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    if B.moe_get_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+    ms_step = ms_total / K
+    tokens_per_s = world * cfg.T / (ms_step / 1e3)
+
+    flops = layer_flops(cfg)
+    gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
+    fp8_peak = 2.0 * peaks["bf16"]          # dense FP8 = 2x dense BF16 (nominal ratio)
+    achieved_tf = flops / gemm_avg_s / 1e12
+    layer_tf = flops / (ms_step / 1e3) / 1e12
+
+    # end to end through the public API: pinned host u in, h' out, every step
+    u_host = u.cpu().pin_memory()
+    out_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
+    u_dev = torch.empty_like(u)
+    b.copy_(b0)
+    for _ in range(2):
+        layer.forward_host(u_host, e, b, out_host, u_dev)
+    torch.cuda.synchronize(dev)
+    Ke = max(3, K // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        layer.forward_host(u_host, e, b, out_host, u_dev)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / Ke
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_tps = world * cfg.T / (e2e_ms / 1e3)
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tps, dt, desc = time_oracle(cfg, n_tokens=1, steps=3, device=dev)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                   "sample": desc, "seconds_per_step": dt}
+        result = {
+            "metric": METRIC,
+            "value": tokens_per_s,
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "e4m3 (fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r,
+                       "K_r": cfg.K_r, "I": cfg.I, "N_s": 1, "seed": cfg.seed,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: 11.3 GB of expert weights stream every step"},
+            "tflops": layer_tf,
+            "pct_fp8_peak": layer_tf / fp8_peak,
+            "roofline": {"bound": "tensor", "kernel": "moe_grouped_gemm_fp8 (2 launches)",
+                         "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": achieved_tf / fp8_peak, "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 {peaks['bf16']} TF/s x2 (burst)",
+                         "gemm_ms": float(np.mean(gemm_ms))},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_tps, "unit": "tokens/s",
+                    "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
+            "gpu_launches": 10 * K,
+            "clocks": clk.summary(),
+        }
+    return result
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: rank 0 only."""
+    if rank != 0:
+        return None
+    import workloads
+    cfg = workloads.CONFIGS[CONFIG_NAME]
+    n_tokens = 1
+    dev = "cpu"
+    # warm-up steps are part of the same timing helper's preparation
+    from oracle import moe as O
+    import numpy as np
+    tokens = np.arange(n_tokens)
+    u, e, b, quant = _oracle_sample_setup(cfg, tokens, device=dev)
+    for _ in range(args.warmup):
+        O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
+    dt = (time.perf_counter() - t0) / args.steps
+    tps = n_tokens / dt
+    desc = (f"oracle forward on token 0 of the {cfg.name} batch per step ({len(quant)} expert "
+            f"FFNs incl. shared), weights pre-quantised by the oracle (inputs drawn on the CPU)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r,
+                   "K_r": cfg.K_r, "I": cfg.I, "N_s": 1, "sample_tokens": n_tokens},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": _blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+"""Thin Python binding of the C ABI: same names as include/moe_fp8.h, torch
+tensors in, status checked, nothing computed here.
+
+Each function takes CUDA tensors (checked for device, dtype, contiguity and
+shape), passes their device pointers and the current CUDA stream to the
+library, and raises MoEError on a non-OK status. bf16 tensors are passed as
+their raw 16-bit patterns; FP8 tensors are torch.uint8 holding E4M3 codes.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import MoEError, check  # noqa: F401
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _want(t, dtype, shape, name):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _opt(t, dtype, shape, name):
+    return None if t is None else _want(t, dtype, shape, name)
+
+
+def moe_quant_1x128(x, q, scale, stream=None):
+    rows, cols = x.shape
+    _want(x, torch.bfloat16, (rows, cols), "x")
+    _want(q, torch.uint8, (rows, cols), "q")
+    _want(scale, torch.float32, (rows, cols // 128), "scale")
+    check("moe_quant_1x128", _lib.load().moe_quant_1x128(
+        _ptr(x), rows, cols, _ptr(q), _ptr(scale), _stream(stream)))
+
+
+def moe_quant_128x128(w, q, scale, stream=None):
+    rows, cols = w.shape
+    _want(w, torch.float32, (rows, cols), "w")
+    _want(q, torch.uint8, (rows, cols), "q")
+    _want(scale, torch.float32, (rows // 128, cols // 128), "scale")
+    check("moe_quant_128x128", _lib.load().moe_quant_128x128(
+        _ptr(w), rows, cols, _ptr(q), _ptr(scale), _stream(stream)))
+
+
+def moe_route(u, e, b, K_r, topk_idx, gates, scores_in=None, scores_out=None, stream=None):
+    N_r = b.shape[0]
+    if scores_in is not None:
+        T = scores_in.shape[0]
+        d = 0
+        _want(scores_in, torch.float32, (T, N_r), "scores_in")
+    else:
+        T, d = u.shape
+        _want(u, torch.bfloat16, (T, d), "u")
+        _want(e, torch.bfloat16, (N_r, d), "e")
+    _want(b, torch.float32, (N_r,), "b")
+    _want(topk_idx, torch.int32, (T, K_r), "topk_idx")
+    _want(gates, torch.float32, (T, K_r), "gates")
+    _opt(scores_out, torch.float32, (T, N_r), "scores_out")
+    check("moe_route", _lib.load().moe_route(
+        _ptr(u), _ptr(e), _ptr(b), _ptr(scores_in), T, d, N_r, K_r, _ptr(scores_out),
+        _ptr(topk_idx), _ptr(gates), _stream(stream)))
+
+
+def moe_permute_workspace(T, N_r):
+    return int(_lib.load().moe_permute_workspace(T, N_r))
+
+
+def moe_permute(topk_idx, N_r, counts, offsets, sorted_token, inv, workspace,
+                xq=None, xs=None, xq_perm=None, xs_perm=None, stream=None):
+    T, K_r = topk_idx.shape
+    _want(topk_idx, torch.int32, (T, K_r), "topk_idx")
+    _want(counts, torch.int32, (N_r,), "counts")
+    _want(offsets, torch.int32, (N_r + 1,), "offsets")
+    _want(sorted_token, torch.int32, (T * K_r,), "sorted_token")
+    _want(inv, torch.int32, (T, K_r), "inv")
+    d = 0
+    if xq is not None:
+        d = xq.shape[1]
+        _want(xq, torch.uint8, (T, d), "xq")
+        _want(xs, torch.float32, (T, d // 128), "xs")
+        _want(xq_perm, torch.uint8, (T * K_r, d), "xq_perm")
+        _want(xs_perm, torch.float32, (T * K_r, d // 128), "xs_perm")
+    check("moe_permute", _lib.load().moe_permute(
+        _ptr(topk_idx), T, K_r, N_r, _ptr(xq), _ptr(xs), d, _ptr(counts), _ptr(offsets),
+        _ptr(sorted_token), _ptr(inv), _ptr(xq_perm), _ptr(xs_perm), _ptr(workspace),
+        workspace.numel() * workspace.element_size() if workspace is not None else 0,
+        _stream(stream)))
+
+
+def moe_grouped_gemm_fp8_workspace(T, K_r, d, I):
+    return int(_lib.load().moe_grouped_gemm_fp8_workspace(T, K_r, d, I))
+
+
+def moe_grouped_gemm_fp8(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down,
+                         s_gate, s_up, s_down, y_perm, y_shared, workspace, stream=None):
+    T, d = xq.shape
+    P = xq_perm.shape[0]
+    G, I, _ = w_gate.shape
+    N_r = G - 1
+    K_r = P // T if T else 0
+    _want(xq_perm, torch.uint8, (P, d), "xq_perm")
+    _want(xs_perm, torch.float32, (P, d // 128), "xs_perm")
+    _want(offsets, torch.int32, (N_r + 1,), "offsets")
+    _want(xq, torch.uint8, (T, d), "xq")
+    _want(xs, torch.float32, (T, d // 128), "xs")
+    _want(w_gate, torch.uint8, (G, I, d), "w_gate")
+    _want(w_up, torch.uint8, (G, I, d), "w_up")
+    _want(w_down, torch.uint8, (G, d, I), "w_down")
+    _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
+    _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
+    _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
+    _want(y_perm, torch.bfloat16, (P, d), "y_perm")
+    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
+    if T and P != T * K_r:
+        raise ValueError("xq_perm rows must be T * K_r")
+    check("moe_grouped_gemm_fp8", _lib.load().moe_grouped_gemm_fp8(
+        _ptr(xq_perm), _ptr(xs_perm), _ptr(offsets), N_r, K_r, _ptr(xq), _ptr(xs), T,
+        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(s_gate), _ptr(s_up), _ptr(s_down),
+        d, I, _ptr(y_perm), _ptr(y_shared), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
+    T, d = u.shape
+    K_r = inv.shape[1]
+    _want(u, torch.bfloat16, (T, d), "u")
+    _want(y_perm, torch.bfloat16, (T * K_r, d), "y_perm")
+    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
+    _want(inv, torch.int32, (T, K_r), "inv")
+    _want(gates, torch.float32, (T, K_r), "gates")
+    _want(out, torch.bfloat16, (T, d), "out")
+    check("moe_combine", _lib.load().moe_combine(
+        _ptr(u), _ptr(y_perm), _ptr(y_shared), _ptr(inv), _ptr(gates), T, K_r, d, _ptr(out),
+        _stream(stream)))
+
+
+def moe_bias_update(b, counts, T, K_r, gamma=0.001, max_over_mean=None, stream=None):
+    N_r = b.shape[0]
+    _want(b, torch.float32, (N_r,), "b")
+    _want(counts, torch.int32, (N_r,), "counts")
+    _opt(max_over_mean, torch.float32, (1,), "max_over_mean")
+    check("moe_bias_update", _lib.load().moe_bias_update(
+        _ptr(b), _ptr(counts), N_r, T, K_r, ctypes.c_float(gamma), _ptr(max_over_mean),
+        _stream(stream)))
+
+
+def moe_debug_wait_timeout(timeout_us, stream=None):
+    check("moe_debug_wait_timeout", _lib.load().moe_debug_wait_timeout(timeout_us, _stream(stream)))
+
+
+def moe_get_error() -> int:
+    st = ctypes.c_int(0)
+    check("moe_get_error", _lib.load().moe_get_error(ctypes.byref(st)))
+    return st.value

@@ -1,0 +1,168 @@
+// Combine (h'_t = u_t + FFN^(s)(u_t) + sum_k g_{t,k} FFN^(r)(u_t)), the
+// auxiliary-loss-free bias update ("DeepSeek-V3 Teknik Raporu", Yöntem 2), and
+// the library's error-word entry points.
+#include "host.cuh"
+
+namespace moe {
+
+// One block per token; each thread handles 8 consecutive channels (16 bytes
+// of bf16) per step. FP32 sum in the fixed order: u, shared, k = 0..K-1.
+__global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ u,
+                                                      const uint16_t* __restrict__ y_perm,
+                                                      const uint16_t* __restrict__ y_shared,
+                                                      const int32_t* __restrict__ inv,
+                                                      const float* __restrict__ gates, int K,
+                                                      int d, int P, uint16_t* out) {
+  __shared__ int s_row[16];
+  __shared__ float s_g[16];
+  const int t = blockIdx.x;
+  if (threadIdx.x < K) {
+    int r = inv[static_cast<size_t>(t) * K + threadIdx.x];
+    if (r < 0 || r >= P) {
+      set_device_error(MOE_ERR_INVALID_ARG);
+      r = -1;
+    }
+    s_row[threadIdx.x] = r;
+    s_g[threadIdx.x] = gates[static_cast<size_t>(t) * K + threadIdx.x];
+  }
+  __syncthreads();
+  const size_t base = static_cast<size_t>(t) * d;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    const uint4 a = *reinterpret_cast<const uint4*>(u + base + c);
+    const uint4 sh = __ldg(reinterpret_cast<const uint4*>(y_shared + base + c));
+    float acc[8];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t sw[4] = {sh.x, sh.y, sh.z, sh.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[2 * i] = bf16_bits_to_float(aw[i] & 0xFFFF) + bf16_bits_to_float(sw[i] & 0xFFFF);
+      acc[2 * i + 1] = bf16_bits_to_float(aw[i] >> 16) + bf16_bits_to_float(sw[i] >> 16);
+    }
+    for (int k = 0; k < K; ++k) {
+      const int r = s_row[k];
+      if (r < 0) continue;
+      const float g = s_g[k];
+      const uint4 y = __ldg(reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(r) * d + c));
+      const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = fmaf(g, bf16_bits_to_float(yw[i] & 0xFFFF), acc[2 * i]);
+        acc[2 * i + 1] = fmaf(g, bf16_bits_to_float(yw[i] >> 16), acc[2 * i + 1]);
+      }
+    }
+    uint4 o;
+    o.x = float_to_bf16_bits(acc[0]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[1])) << 16);
+    o.y = float_to_bf16_bits(acc[2]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[3])) << 16);
+    o.z = float_to_bf16_bits(acc[4]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[5])) << 16);
+    o.w = float_to_bf16_bits(acc[6]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[7])) << 16);
+    *reinterpret_cast<uint4*>(out + base + c) = o;
+  }
+}
+
+// One block: b_i -= gamma if counts_i * N_r > T*K_r, b_i += gamma if below,
+// unchanged if equal (FP32 arithmetic). Also max_i counts_i * N_r / (T*K_r).
+__global__ void __launch_bounds__(1024) bias_update_kernel(float* b, const int32_t* __restrict__ counts,
+                                                           int N_r, long long mean_load_x_nr,
+                                                           float gamma, float* max_over_mean) {
+  __shared__ int s_max[32];
+  int local_max = 0;
+  for (int i = threadIdx.x; i < N_r; i += blockDim.x) {
+    const int c = counts[i];
+    const long long load = static_cast<long long>(c) * N_r;
+    if (load > mean_load_x_nr)
+      b[i] = b[i] - gamma;
+    else if (load < mean_load_x_nr)
+      b[i] = b[i] + gamma;
+    local_max = max(local_max, c);
+  }
+  if (max_over_mean == nullptr) return;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) local_max = max(local_max, __shfl_xor_sync(0xffffffffu, local_max, o));
+  if (lane_id() == 0) s_max[threadIdx.x >> 5] = local_max;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int m = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) m = max(m, s_max[w]);
+    *max_over_mean = mean_load_x_nr > 0
+                         ? static_cast<float>(static_cast<double>(m) * N_r / static_cast<double>(mean_load_x_nr))
+                         : 0.0f;
+  }
+}
+
+// Waits on an mbarrier nothing signals; gives up after limit_ns.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
+}  // namespace moe
+
+extern "C" int moe_combine(const uint16_t* u, const uint16_t* y_perm, const uint16_t* y_shared,
+                           const int32_t* inv, const float* gates, int T, int K_r, int d,
+                           uint16_t* out, void* stream) {
+  using namespace moe;
+  MOE_CHECK_ARG(T >= 0 && K_r >= 1 && d >= 0);
+  MOE_CHECK_SUPPORTED(K_r <= 16 && d % 8 == 0);
+  if (T == 0 || d == 0) return MOE_OK;
+  MOE_CHECK_ARG(u && y_perm && y_shared && inv && gates && out);
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(u) % 16 == 0 && reinterpret_cast<uintptr_t>(y_perm) % 16 == 0 &&
+                reinterpret_cast<uintptr_t>(y_shared) % 16 == 0 && reinterpret_cast<uintptr_t>(out) % 16 == 0);
+  MOE_CHECK_SUPPORTED(static_cast<long long>(T) * K_r < (1LL << 31));
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  combine_kernel<<<T, 128, 0, as_stream(stream)>>>(u, y_perm, y_shared, inv, gates, K_r, d, T * K_r, out);
+  return launch_status();
+}
+
+extern "C" int moe_bias_update(float* b, const int32_t* counts, int N_r, int T, int K_r, float gamma,
+                               float* max_over_mean_out, void* stream) {
+  using namespace moe;
+  MOE_CHECK_ARG(N_r >= 1 && T >= 0 && K_r >= 1 && b && counts);
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  bias_update_kernel<<<1, 1024, 0, as_stream(stream)>>>(b, counts, N_r, static_cast<long long>(T) * K_r,
+                                                        gamma, max_over_mean_out);
+  return launch_status();
+}
+
+extern "C" int moe_debug_wait_timeout(int timeout_us, void* stream) {
+  using namespace moe;
+  MOE_CHECK_ARG(timeout_us >= 1 && timeout_us <= 1000000);
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  wait_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(timeout_us) * 1000ull);
+  return launch_status();
+}
+
+extern "C" int moe_get_error(int* device_status) {
+  using namespace moe;
+  MOE_CHECK_ARG(device_status);
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  *device_status = v;
+  return MOE_OK;
+}
+
+extern "C" const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE";
+    default: return "unknown moe_status";
+  }
+}
+
+extern "C" int moe_version(void) { return 100; }

@@ -1,0 +1,477 @@
+// Grouped FP8 GEMM for all expert FFNs of the layer (routed experts on the
+// permuted rows, the shared expert on all tokens).
+//
+// Numerics ("DeepSeek-V3 Teknik Raporu", Temel fikirler, FP8 bullet: E4M3
+// operands, 1x128 activation tiles, 128x128 weight blocks, FP32 promotion of
+// the accumulation every N_c = 128): every product is
+//     C[m, n] = sum_kb  s_A[m, kb] * s_W[n/128, kb] * P_kb[m, n],
+//     P_kb = A[m, kb*128 : kb*128+128] . W[n, kb*128 : kb*128+128],
+// The tensor cores produce each 128-wide partial P_kb into a fresh TMEM
+// buffer (four tcgen05.mma kind::f8f6f4 of K = 32). The epilogue warps read it
+// with tcgen05.ld, multiply by the two FP32 scales and add it to an FP32
+// register accumulator. Only one K block ever sums inside the tensor core. On
+// H800 the promotion moved the partial sums into CUDA-core registers; here
+// TMEM plays that role with two partial buffers in flight, so the next block's
+// MMAs overlap the FMAs of the current one.
+//
+// Structure (one persistent CTA per SM, 320 threads):
+//   warp 0    TMA producer: A tile 128 x 128 and B tile 256 x 128 per K block
+//             (128-byte swizzle), 4-stage ring.
+//   warp 1    MMA issuer (one thread) and TMEM owner (512 columns = 2 x 256).
+//   warps 2-9 epilogue: warp w reads TMEM lanes 32*(w%4).. (rows), and
+//             (w-2)/4 selects the column half.
+//
+// Two launches:
+//   phase 1: per tile (group g, 128 rows, 128 intermediate channels n):
+//            B = [W_gate rows n*128..+128 ; W_up rows n*128..+128], N = 256.
+//            Epilogue: SwiGLU a = silu(G) * U, 1x128 requantisation to E4M3
+//            (the tile is exactly one 128-channel scale tile), written to H.
+//   phase 2: per tile (group g, 128 rows, 256 output channels):
+//            A = H, B = W_down rows, epilogue converts to bf16.
+// Tiles are numbered group-major (shared expert last), then row tile, then
+// column tile, and dealt round-robin to CTAs, so the CTAs running at the same
+// time share weight tiles and activation rows through L2.
+#include "host.cuh"
+
+namespace moe {
+namespace gg {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 320;
+constexpr int EPI_THREADS = 256;
+constexpr int MAX_GROUPS = 1025;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct Args {
+  const int32_t* offsets;
+  int N_r, T, P, d, I;
+  const float* xs_perm;
+  const float* xs;
+  const float* s_gate;
+  const float* s_up;
+  const float* s_down;
+  uint8_t* H;
+  float* Hs;
+  uint16_t* y_perm;
+  uint16_t* y_shared;
+};
+
+struct Smem {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint64_t xbar;      // epilogue exchange of per-half max-abs (phase 1)
+  uint32_t tmem_base;
+  int abort;
+  int total_tiles;
+  int off[MAX_GROUPS + 1];
+  int tile_start[MAX_GROUPS + 1];
+  float amax_x[2][2][BM];  // [tile parity][column half][row]
+};
+
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Smem);
+
+__device__ __forceinline__ int find_group(const int* start, int G, int t) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+struct Tile {
+  int g, m, n, rows, row0;  // rows of the group; row0 = first row of the group in its A tensor
+  bool shared;
+};
+
+template <int PHASE>
+__device__ __forceinline__ Tile decode_tile(const Smem& sm, const Args& a, int t, int n_tiles) {
+  Tile tl;
+  const int G = a.N_r + 1;
+  tl.g = find_group(sm.tile_start, G, t);
+  const int local = t - sm.tile_start[tl.g];
+  tl.m = local / n_tiles;
+  tl.n = local - tl.m * n_tiles;
+  tl.shared = tl.g == a.N_r;
+  if (tl.shared) {
+    tl.rows = a.T;
+    tl.row0 = PHASE == 1 ? 0 : a.P;  // phase 2 reads H, where shared rows follow the routed ones
+  } else {
+    tl.row0 = sm.off[tl.g];
+    tl.rows = sm.off[tl.g + 1] - tl.row0;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ float silu(float x) { return __fdiv_rn(x, 1.0f + expf(-x)); }
+
+template <int PHASE>
+__global__ void __maxnreg__(200)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                        const Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>(tiles + STAGES * STAGE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+  const int G = a.N_r + 1;
+  const int KB = (PHASE == 1 ? a.d : a.I) / BK;            // K blocks per tile
+  const int n_tiles = PHASE == 1 ? a.I / 128 : a.d / BN;    // column tiles per row tile
+
+  // ---- setup: barriers, TMEM, the tile table
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.tfull[b], 1);
+      mbar_init(&sm.tempty[b], EPI_THREADS / 32);
+    }
+    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.xbar, EPI_THREADS);
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_b0);
+    tma_prefetch_desc(&tm_b1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i <= a.N_r; i += THREADS) sm.off[i] = a.offsets[i];
+  __syncthreads();
+  for (int g = threadIdx.x; g < G; g += THREADS) {
+    const int rows = g == a.N_r ? a.T : sm.off[g + 1] - sm.off[g];
+    sm.tile_start[g] = ((rows + BM - 1) / BM) * n_tiles;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive prefix sum of tile counts, in place
+    int carry = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int i = base + lane;
+      const int v = i < G ? sm.tile_start[i] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      if (i < G) sm.tile_start[i] = carry + incl - v;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      sm.tile_start[G] = carry;
+      sm.total_tiles = carry;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const int total = sm.total_tiles;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int armed[STAGES];
+      for (int s = 0; s < STAGES; ++s) armed[s] = -1;
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint64_t pol_w = l2_policy_evict_last();
+      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
+        const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
+        const CUtensorMap* am = (PHASE == 1 && tl.shared) ? &tm_x : &tm_a;
+        const int arow = tl.row0 + tl.m * BM;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) break;
+          uint8_t* dst = tiles + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&sm.full[stage], STAGE_BYTES);
+          tma_load_2d(dst, am, &sm.full[stage], kb * BK, arow);
+          if (PHASE == 1) {
+            const int wrow = tl.g * a.I + tl.n * 128;
+            tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+            tma_load_2d_hint(dst + A_BYTES + B_BYTES / 2, &tm_b1, &sm.full[stage], kb * BK, wrow, pol_w);
+          } else {
+            const int wrow = tl.g * a.d + tl.n * BN;
+            tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+          }
+          armed[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort) {
+        volatile int never = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s] >= 0) mbar_wait(&sm.full[s], armed[s], &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(0, 0, BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t tphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) { ok = false; break; }
+          if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
+          const uint64_t ad = sw128_kmajor_desc(a_addr);
+          const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
+          const uint32_t d_tmem = tmem + buf * BN;
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k) umma_f8f6f4(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0);
+          umma_commit(&sm.empty[stage]);
+          umma_commit(&sm.tfull[buf]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+          buf ^= 1;
+          if (buf == 0) tphase ^= 1;
+        }
+      }
+      umma_commit(&sm.drain);
+      volatile int never = 0;
+      mbar_wait(&sm.drain, 0, &never, 100000000ull);
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    int buf = 0;
+    uint32_t tphase = 0;
+    uint32_t xpar = 0;
+    const int KBd = a.d / BK, KBi = a.I / BK;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
+      const int rr = tl.m * BM + r;          // row within the group
+      const bool valid = rr < tl.rows;
+      const int grow = tl.row0 + rr;         // row in the A tensor (and its scales)
+      const float* sa_ptr;
+      const float* sb0;
+      const float* sb1;
+      if (PHASE == 1) {
+        sa_ptr = (tl.shared ? a.xs : a.xs_perm) + static_cast<size_t>(grow) * KBd;
+        sb0 = a.s_gate + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
+        sb1 = a.s_up + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
+      } else {
+        sa_ptr = a.Hs + static_cast<size_t>(grow) * KBi;
+        sb0 = a.s_down + static_cast<size_t>(tl.g * KBd + tl.n * 2 + half) * KBi;
+        sb1 = sb0;
+      }
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      float sa_n = valid ? __ldg(sa_ptr) : 0.0f;
+      float s0_n = __ldg(sb0), s1_n = __ldg(sb1);
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        const float sa = sa_n, s0 = s0_n, s1 = s1_n;
+        if (kb + 1 < KB) {  // next block's scales, loaded one block ahead
+          sa_n = valid ? __ldg(sa_ptr + kb + 1) : 0.0f;
+          s0_n = __ldg(sb0 + kb + 1);
+          s1_n = __ldg(sb1 + kb + 1);
+        }
+        if (!warp_wait(&sm.tfull[buf], tphase, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ta = tmem + lane_base + buf * BN;
+        float v[32];
+        if (PHASE == 1) {
+          const float fg = sa * s0, fu = sa * s1;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(ta + half * 64 + c * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(fg, v[j], acc[c * 32 + j]);
+          }
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld32(ta + 128 + half * 64 + c * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[64 + c * 32 + j] = fmaf(fu, v[j], acc[64 + c * 32 + j]);
+          }
+        } else {
+          const float f = sa * s0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(ta + half * 128 + c * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(f, v[j], acc[c * 32 + j]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+        buf ^= 1;
+        if (buf == 0) tphase ^= 1;
+      }
+      if (!ok) break;
+
+      if (PHASE == 1) {
+        // SwiGLU on this thread's 64 channels, then the 1x128 requantisation
+        // whose max-abs spans both column halves (the partner warp).
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float x = silu(acc[j]) * acc[64 + j];
+          acc[j] = x;
+          amax = fmaxf(amax, fabsf(x));
+        }
+        // exchange through shared memory, double-buffered by tile parity; the
+        // mbarrier wait is bounded like every other wait here
+        sm.amax_x[xpar][half][r] = amax;
+        mbar_arrive(&sm.xbar);
+        if (!warp_wait(&sm.xbar, xpar, abort)) break;
+        amax = fmaxf(amax, sm.amax_x[xpar][half ^ 1][r]);
+        xpar ^= 1;
+        const float s = tile_scale(amax);
+        if (valid) {
+          const size_t hrow = static_cast<size_t>(tl.shared ? a.P + rr : tl.row0 + rr);
+          uint4* dst = reinterpret_cast<uint4*>(a.H + hrow * a.I + tl.n * 128 + half * 64);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int j = i * 16 + k * 4;
+              w[k] = e4m3x2(__fdiv_rn(acc[j], s), __fdiv_rn(acc[j + 1], s)) |
+                     (e4m3x2(__fdiv_rn(acc[j + 2], s), __fdiv_rn(acc[j + 3], s)) << 16);
+            }
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          if (half == 0) a.Hs[hrow * KBi + tl.n] = s;
+        }
+      } else {
+        if (valid) {
+          uint16_t* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
+                                     : a.y_perm + static_cast<size_t>(tl.row0 + rr) * a.d;
+          uint4* dst = reinterpret_cast<uint4*>(yrow + tl.n * BN + half * 128);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              w[k] = float_to_bf16_bits(acc[i * 8 + 2 * k]) |
+                     (static_cast<uint32_t>(float_to_bf16_bits(acc[i * 8 + 2 * k + 1])) << 16);
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace gg
+}  // namespace moe
+
+extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
+  (void)d;
+  if (T <= 0 || K_r <= 0 || I <= 0) return 0;
+  const size_t rows = static_cast<size_t>(T) * K_r + T;
+  return moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float);
+}
+
+extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
+                                    int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
+                                    const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
+                                    const float* s_gate, const float* s_up, const float* s_down, int d,
+                                    int I, uint16_t* y_perm, uint16_t* y_shared, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  using namespace moe;
+  using namespace moe::gg;
+  MOE_CHECK_ARG(N_r >= 1 && K_r >= 1 && T >= 0 && d > 0 && I > 0);
+  MOE_CHECK_SUPPORTED(N_r + 1 <= MAX_GROUPS && K_r <= N_r && d % 256 == 0 && I % 128 == 0);
+  const long long P = static_cast<long long>(T) * K_r;
+  MOE_CHECK_SUPPORTED(P + T < (1LL << 31) && static_cast<long long>(N_r + 1) * (d > I ? d : I) < (1LL << 31));
+  if (T == 0) return MOE_OK;
+  MOE_CHECK_ARG(xq_perm && xs_perm && offsets && xq && xs && w_gate && w_up && w_down && s_gate && s_up &&
+                s_down && y_perm && y_shared && workspace);
+  MOE_CHECK_ARG(ws_bytes >= moe_grouped_gemm_fp8_workspace(T, K_r, d, I));
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(workspace) % 256 == 0 && reinterpret_cast<uintptr_t>(y_perm) % 16 == 0 &&
+                reinterpret_cast<uintptr_t>(y_shared) % 16 == 0);
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  cudaStream_t s = as_stream(stream);
+
+  const long long rowsH = P + T;
+  uint8_t* H = static_cast<uint8_t*>(workspace);
+  float* Hs = reinterpret_cast<float*>(H + align256(static_cast<size_t>(rowsH) * I));
+
+  CUtensorMap tmA, tmX, tmWg, tmWu, tmH, tmWd;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  if (int st = make_tmap_2d(&tmA, xq_perm, U8, 1, P, d, BM, BK)) return st;
+  if (int st = make_tmap_2d(&tmX, xq, U8, 1, T, d, BM, BK)) return st;
+  if (int st = make_tmap_2d(&tmWg, w_gate, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
+  if (int st = make_tmap_2d(&tmWu, w_up, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
+  if (int st = make_tmap_2d(&tmH, H, U8, 1, rowsH, I, BM, BK)) return st;
+  if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
+
+  Args args;
+  args.offsets = offsets;
+  args.N_r = N_r;
+  args.T = T;
+  args.P = static_cast<int>(P);
+  args.d = d;
+  args.I = I;
+  args.xs_perm = xs_perm;
+  args.xs = xs;
+  args.s_gate = s_gate;
+  args.s_up = s_up;
+  args.s_down = s_down;
+  args.H = H;
+  args.Hs = Hs;
+  args.y_perm = y_perm;
+  args.y_shared = y_shared;
+
+  // upper bound on row tiles: every non-empty routed group wastes < 1 tile
+  const long long m_tiles = (P + BM - 1) / BM + (P < N_r ? P : N_r) + (T + BM - 1) / BM;
+  const long long t1 = m_tiles * (I / 128), t2 = m_tiles * (d / BN);
+  const int g1 = static_cast<int>(t1 < di.sm_count ? t1 : di.sm_count);
+  const int g2 = static_cast<int>(t2 < di.sm_count ? t2 : di.sm_count);
+
+  auto k1 = grouped_gemm_kernel<1>;
+  auto k2 = grouped_gemm_kernel<2>;
+  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)) != cudaSuccess ||
+      cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  k1<<<g1, THREADS, SMEM_BYTES, s>>>(tmA, tmX, tmWg, tmWu, args);
+  if (int st = launch_status()) return st;
+  k2<<<g2, THREADS, SMEM_BYTES, s>>>(tmH, tmH, tmWd, tmWd, args);
+  return launch_status();
+}

@@ -1,0 +1,99 @@
+"""MoELayerFP8: owns the device buffers of one DeepSeekMoE FP8 layer and runs
+its forward pass through the C ABI, step by step:
+
+  route -> quant_1x128 -> permute -> grouped FP8 GEMM (routed + shared)
+        -> combine -> bias update
+
+("DeepSeek-V3 Teknik Raporu", Yöntem 2 for the layer equations; Temel
+fikirler, FP8 bullet for the quantisation scheme). PyTorch only allocates
+memory and provides the stream; every step runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class MoELayerFP8:
+    def __init__(self, T: int, d: int, N_r: int, K_r: int, I: int, device="cuda"):
+        self.T, self.d, self.N_r, self.K_r, self.I = T, d, N_r, K_r, I
+        self.device = torch.device(device)
+        G, P = N_r + 1, T * K_r
+        dev = dict(device=self.device)
+        u8, f32, i32, bf = torch.uint8, torch.float32, torch.int32, torch.bfloat16
+        # weights: slot N_r is the shared expert
+        self.w_gate = torch.empty(G, I, d, dtype=u8, **dev)
+        self.w_up = torch.empty(G, I, d, dtype=u8, **dev)
+        self.w_down = torch.empty(G, d, I, dtype=u8, **dev)
+        self.s_gate = torch.empty(G, I // 128, d // 128, dtype=f32, **dev)
+        self.s_up = torch.empty(G, I // 128, d // 128, dtype=f32, **dev)
+        self.s_down = torch.empty(G, d // 128, I // 128, dtype=f32, **dev)
+        # activations
+        self.topk_idx = torch.empty(T, K_r, dtype=i32, **dev)
+        self.gates = torch.empty(T, K_r, dtype=f32, **dev)
+        self.xq = torch.empty(T, d, dtype=u8, **dev)
+        self.xs = torch.empty(T, d // 128, dtype=f32, **dev)
+        self.counts = torch.empty(N_r, dtype=i32, **dev)
+        self.offsets = torch.empty(N_r + 1, dtype=i32, **dev)
+        self.sorted_token = torch.empty(P, dtype=i32, **dev)
+        self.inv = torch.empty(T, K_r, dtype=i32, **dev)
+        self.xq_perm = torch.empty(P, d, dtype=u8, **dev)
+        self.xs_perm = torch.empty(P, d // 128, dtype=f32, **dev)
+        self.y_perm = torch.empty(P, d, dtype=bf, **dev)
+        self.y_shared = torch.empty(T, d, dtype=bf, **dev)
+        self.out = torch.empty(T, d, dtype=bf, **dev)
+        self.max_over_mean = torch.zeros(1, dtype=f32, **dev)
+        self.ws_perm = torch.empty(max(B.moe_permute_workspace(T, N_r), 16), dtype=u8, **dev)
+        self.ws_gemm = torch.empty(max(B.moe_grouped_gemm_fp8_workspace(T, K_r, d, I), 256),
+                                   dtype=u8, **dev)
+
+    # ---------------------------------------------------------------- weights
+    def load_expert(self, slot: int, w_gate: torch.Tensor, w_up: torch.Tensor,
+                    w_down: torch.Tensor, stream=None) -> None:
+        """Quantises one expert's FP32 weights (on the device) into slot `slot`."""
+        B.moe_quant_128x128(w_gate, self.w_gate[slot], self.s_gate[slot], stream)
+        B.moe_quant_128x128(w_up, self.w_up[slot], self.s_up[slot], stream)
+        B.moe_quant_128x128(w_down, self.w_down[slot], self.s_down[slot], stream)
+
+    # ---------------------------------------------------------------- steps
+    def route(self, u, e, b, scores_out=None, stream=None):
+        B.moe_route(u, e, b, self.K_r, self.topk_idx, self.gates, scores_out=scores_out,
+                    stream=stream)
+
+    def quant(self, u, stream=None):
+        B.moe_quant_1x128(u, self.xq, self.xs, stream)
+
+    def permute(self, stream=None):
+        B.moe_permute(self.topk_idx, self.N_r, self.counts, self.offsets, self.sorted_token,
+                      self.inv, self.ws_perm, self.xq, self.xs, self.xq_perm, self.xs_perm,
+                      stream=stream)
+
+    def experts(self, stream=None):
+        B.moe_grouped_gemm_fp8(self.xq_perm, self.xs_perm, self.offsets, self.xq, self.xs,
+                               self.w_gate, self.w_up, self.w_down, self.s_gate, self.s_up,
+                               self.s_down, self.y_perm, self.y_shared, self.ws_gemm, stream)
+
+    def combine(self, u, stream=None):
+        B.moe_combine(u, self.y_perm, self.y_shared, self.inv, self.gates, self.out, stream)
+
+    def bias_update(self, b, gamma=0.001, stream=None):
+        B.moe_bias_update(b, self.counts, self.T, self.K_r, gamma, self.max_over_mean, stream)
+
+    def forward(self, u, e, b, update_bias=True, stream=None):
+        """One pass of the layer on device tensors; returns self.out."""
+        self.route(u, e, b, stream=stream)
+        self.quant(u, stream)
+        self.permute(stream)
+        self.experts(stream)
+        self.combine(u, stream)
+        if update_bias:
+            self.bias_update(b, stream=stream)
+        return self.out
+
+    def forward_host(self, u_host, e, b, out_host, u_dev, update_bias=True, stream=None):
+        """End to end from pinned host memory: copy u in, run, copy h' out."""
+        u_dev.copy_(u_host, non_blocking=True)
+        self.forward(u_dev, e, b, update_bias, stream)
+        out_host.copy_(self.out, non_blocking=True)
+        return out_host

@@ -1,0 +1,223 @@
+/*
+ * moe_fp8.h - C ABI of the DeepSeekMoE FP8 layer forward pass on B200 (sm_100a).
+ *
+ * The layer (one MoE FFN of DeepSeek-V3) computes, for every token t,
+ *
+ *   h'_t = u_t + FFN^(s)(u_t) + sum_{i=1..N_r} g_{i,t} FFN^(r)_i(u_t)
+ *   s_{i,t} = Sigmoid(u_t . e_i)
+ *   g'_{i,t} = s_{i,t} if s_{i,t} + b_i is among the K_r largest of {s_{j,t} + b_j}, else 0
+ *   g_{i,t}  = g'_{i,t} / sum_j g'_{j,t}
+ *   b_i <- b_i - gamma (expert i overloaded) / b_i + gamma (underloaded), gamma = 0.001
+ *
+ * as printed in "DeepSeek-V3 Teknik Raporu" (xyznot.com/tr/paper/2412.19437),
+ * section "Yöntem", part 2 "Yardımcı Kayıpsız Dengelemeli DeepSeekMoE", and in
+ * its French copy "DeepSeek-V3 Technical Report" (xyznot.com/fr), "Méthode" 2.
+ * The expert FFNs run in FP8 E4M3 with one FP32 scale per 1x128 activation tile
+ * and per 128x128 weight block, accumulating in FP32 with the scales applied at
+ * every 128-wide K block (same pages, "Temel fikirler" / "Idées clés", FP8
+ * bullet: "FP8 Karma Duyarlıklı Eğitim").
+ *
+ * Conventions for every call
+ *   - All pointers are DEVICE pointers owned by the caller, unless a comment
+ *     says otherwise. No call allocates memory, and no call synchronises the
+ *     host, except moe_get_error.
+ *   - `stream` is a cudaStream_t passed as void*; work is enqueued on it.
+ *   - Tensors are dense and row-major. bf16 is passed as uint16_t bits.
+ *     FP8 tensors are uint8 E4M3 codes.
+ *   - Activation scales are FP32, row-major [rows][cols/128], one per 1x128
+ *     tile. Weight scales are FP32 [rows/128][cols/128], one per 128x128 block.
+ *   - Expert weights are stacked over N_r + 1 slots; slot N_r is the shared
+ *     expert. W_gate and W_up are [N_r+1][I][d] and W_down is [N_r+1][d][I]
+ *     (K-major: the reduction dimension is contiguous).
+ *   - Every call returns a moe_status. Arguments are checked on the host before
+ *     any launch. A device-side failure (a wait that timed out) is recorded in a
+ *     device error word that moe_get_error reads.
+ *   - Stateless: the routing bias b is caller-owned state.
+ */
+#ifndef MOE_FP8_H
+#define MOE_FP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, workspace too small */
+  MOE_ERR_UNSUPPORTED = 2,   /* a size outside what the kernels handle (see each call) */
+  MOE_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+  MOE_ERR_TIMEOUT = 4,       /* a device wait exceeded its limit (read by moe_get_error) */
+  MOE_ERR_NO_DEVICE = 5      /* no sm_100 device is current */
+} moe_status;
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(int status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+MOE_API int moe_version(void);
+
+/*
+ * moe_get_error: synchronises the device, then reads and clears the device
+ * error word that kernels set when a bounded wait gave up.
+ *   device_status (HOST pointer, out): MOE_OK or MOE_ERR_TIMEOUT.
+ * Returns MOE_OK, or MOE_ERR_CUDA if synchronising failed.
+ */
+MOE_API int moe_get_error(int* device_status);
+
+/*
+ * moe_quant_1x128: activation quantisation, one FP32 scale per 1x128 tile
+ * ("DeepSeek-V3 Teknik Raporu", Temel fikirler, FP8 bullet: 1x128 tile-wise
+ * activation scaling, E4M3).
+ *   x      [rows][cols] bf16 (input)
+ *   q      [rows][cols] E4M3 (output)
+ *   scale  [rows][cols/128] FP32 (output)
+ * Per tile: amax = max |x|, scale = fl32(amax / 448) (1 if that is zero),
+ * q = E4M3 round-to-nearest-even, saturating, of fl32(x / scale).
+ * cols must be a multiple of 128 (else MOE_ERR_UNSUPPORTED); rows may be 0.
+ */
+MOE_API int moe_quant_1x128(const uint16_t* x, int rows, int cols, uint8_t* q,
+                    float* scale, void* stream);
+
+/*
+ * moe_quant_128x128: weight quantisation, one FP32 scale per 128x128 block
+ * (same passage: 128x128 block-wise weight scaling). Same scale rule as above.
+ *   w      [rows][cols] FP32 (input)
+ *   q      [rows][cols] E4M3 (output)
+ *   scale  [rows/128][cols/128] FP32 (output)
+ * rows and cols must be multiples of 128.
+ */
+MOE_API int moe_quant_128x128(const float* w, int rows, int cols, uint8_t* q,
+                      float* scale, void* stream);
+
+/*
+ * moe_route: the router ("DeepSeek-V3 Teknik Raporu", Yöntem 2: the
+ * s_{i,t}, g'_{i,t} and g_{i,t} equations).
+ *   u          [T][d] bf16 token activations
+ *   e          [N_r][d] bf16 expert centroids
+ *   b          [N_r] FP32 routing bias (only affects selection)
+ *   scores_in  NULL, or [T][N_r] FP32 affinities to use instead of
+ *              Sigmoid(u . e) (u and e are then not read and may be NULL)
+ *   scores_out NULL, or [T][N_r] FP32: the affinities s_{i,t}
+ *   topk_idx   [T][K_r] int32: selected experts, ordered by key s+b
+ *              descending, equal keys by lower index first
+ *   gates      [T][K_r] FP32: g = s_sel / sum(s_sel), in the same order
+ * The logits u . e run on the tensor cores in BF16 with FP32 accumulation; the
+ * key s + b is formed in FP32. Limits: 1 <= K_r <= 16, K_r <= N_r <= 256,
+ * d a multiple of 64.
+ */
+MOE_API int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
+              const float* scores_in, int T, int d, int N_r, int K_r,
+              float* scores_out, int32_t* topk_idx, float* gates,
+              void* stream);
+
+/*
+ * moe_permute_workspace: bytes of scratch moe_permute needs for T tokens and
+ * N_r experts (two int32 tables of ceil(T/256) x N_r).
+ */
+MOE_API size_t moe_permute_workspace(int T, int N_r);
+
+/*
+ * moe_permute: groups the (token, expert) pairs by expert with a stable
+ * counting sort (histogram, prefix sum, scatter): row p of the permuted
+ * layout holds token sorted_token[p]; rows are ordered by expert, then token.
+ * The pages group tokens per expert without printing how; this is the plain
+ * stable reading.
+ *   topk_idx     [T][K_r] int32, each row distinct experts in [0, N_r)
+ *   xq, xs       NULL, or the token rows to move: [T][d] E4M3, [T][d/128] FP32
+ *   counts       [N_r] int32 (out): rows per expert
+ *   offsets      [N_r+1] int32 (out): exclusive prefix sum of counts
+ *   sorted_token [T*K_r] int32 (out)
+ *   inv          [T][K_r] int32 (out): row of the pair (t, k)
+ *   xq_perm, xs_perm  NULL (when xq is NULL) or [T*K_r][d], [T*K_r][d/128] (out)
+ *   workspace    device scratch of moe_permute_workspace(T, N_r) bytes
+ * Limits: N_r <= 1024, K_r <= 16, d a multiple of 128.
+ */
+MOE_API int moe_permute(const int32_t* topk_idx, int T, int K_r, int N_r,
+                const uint8_t* xq, const float* xs, int d,
+                int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                int32_t* inv, uint8_t* xq_perm, float* xs_perm,
+                void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_grouped_gemm_fp8_workspace: bytes of scratch for the intermediate
+ * H = requant(SwiGLU(...)) of P = T*K_r routed rows plus T shared rows:
+ * (P + T) * I bytes of E4M3 and (P + T) * I/128 FP32 scales.
+ */
+MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
+
+/*
+ * moe_grouped_gemm_fp8: every expert FFN of the layer on FP8 operands.
+ * For routed expert i (rows offsets[i]..offsets[i+1] of xq_perm) and for the
+ * shared expert (slot N_r, all T rows of xq):
+ *   G = X W_gate^T, U = X W_up^T      (FP8 x FP8 -> FP32)
+ *   A = silu(G) * U,  H = quant_1x128(A)
+ *   Y = H W_down^T -> bf16
+ * Each product is sum over 128-wide K blocks kb of
+ *   s_X[m,kb] * s_W[n/128,kb] * (X_kb . W_kb),
+ * the block partial coming from the tensor cores and the scaling and the sum
+ * in FP32 ("Temel fikirler", FP8 bullet: FP32 promotion every N_c = 128).
+ *   xq_perm, xs_perm  [P][d] E4M3, [P][d/128] FP32, P = T*K_r
+ *   offsets           [N_r+1] int32 (device) from moe_permute
+ *   xq, xs            [T][d], [T][d/128]: the shared expert's input
+ *   w_gate, w_up      [N_r+1][I][d] E4M3;  s_gate, s_up  [N_r+1][I/128][d/128]
+ *   w_down            [N_r+1][d][I] E4M3;  s_down        [N_r+1][d/128][I/128]
+ *   y_perm            [P][d] bf16 (out)    y_shared [T][d] bf16 (out)
+ *   workspace         moe_grouped_gemm_fp8_workspace(T, K_r, d, I) bytes
+ * Limits: d a multiple of 256, I a multiple of 128, N_r <= 1024.
+ */
+MOE_API int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm,
+                         const int32_t* offsets, int N_r, int K_r,
+                         const uint8_t* xq, const float* xs, int T,
+                         const uint8_t* w_gate, const uint8_t* w_up,
+                         const uint8_t* w_down, const float* s_gate,
+                         const float* s_up, const float* s_down, int d, int I,
+                         uint16_t* y_perm, uint16_t* y_shared,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
+ * ("DeepSeek-V3 Teknik Raporu", Yöntem 2, the h'_t equation). The sum is FP32
+ * in the fixed order u, shared, k = 0..K_r-1.
+ *   u, y_shared [T][d] bf16;  y_perm [T*K_r][d] bf16;  inv, gates [T][K_r]
+ *   out [T][d] bf16 (may alias u)
+ * d must be a multiple of 8.
+ */
+MOE_API int moe_combine(const uint16_t* u, const uint16_t* y_perm,
+                const uint16_t* y_shared, const int32_t* inv,
+                const float* gates, int T, int K_r, int d, uint16_t* out,
+                void* stream);
+
+/*
+ * moe_bias_update: auxiliary-loss-free balancing ("DeepSeek-V3 Teknik
+ * Raporu", Yöntem 2, last paragraph): b_i -= gamma when expert i is
+ * overloaded, b_i += gamma when underloaded. Overloaded means
+ * counts[i] * N_r > T * K_r (load above the mean); equal load leaves b_i.
+ *   b                  [N_r] FP32, updated in place
+ *   counts             [N_r] int32 from moe_permute
+ *   max_over_mean_out  NULL or [1] FP32 (device): max_i counts[i] * N_r / (T*K_r)
+ */
+MOE_API int moe_bias_update(float* b, const int32_t* counts, int N_r, int T, int K_r,
+                    float gamma, float* max_over_mean_out, void* stream);
+
+/*
+ * moe_debug_wait_timeout: launches one block that waits on a barrier nothing
+ * ever signals, with a limit of timeout_us microseconds; the wait gives up and
+ * records MOE_ERR_TIMEOUT in the device error word. Exists to test the
+ * timeout path without hanging a GPU. 1 <= timeout_us <= 1000000.
+ */
+MOE_API int moe_debug_wait_timeout(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_FP8_H */

@@ -55,38 +55,28 @@ def encode(x: np.ndarray) -> np.ndarray:
     """float64 values -> uint8 E4M3 codes, round-to-nearest-even, satfinite.
 
     Within the binade [2^k, 2^(k+1)) (k >= -6) the representable magnitudes are
-    spaced 2^(k-3); below 2^-6 they are the subnormals n * 2^-9. So the nearest
-    value is rint(|x| / q) * q with q that spacing; numpy's rint rounds ties to
-    the even integer, and the integer's parity is the mantissa's parity (a
-    carry into the next binade lands on mantissa 0, also even).
+    n * 2^(k-3) with n = 8..15 (exponent field k+7, mantissa n-8); below 2^-6
+    they are the subnormals n * 2^-9, n = 0..7 (exponent field 0, mantissa n).
+    So the nearest value has n = rint(|x| / 2^(k-3)); numpy's rint rounds ties
+    to the even integer, and n's parity is the mantissa's parity. n = 16 is the
+    carry into the next binade (mantissa 0, also even); n = 8 from the
+    subnormal range is the smallest normal.
     """
     x = np.asarray(x, dtype=np.float64)
     if np.isnan(x).any():
         raise ValueError("NaN input to the E4M3 encoder")
     neg = np.signbit(x)
-    a = np.abs(x)
-    a = np.minimum(a, E4M3_MAX)                      # satfinite
+    a = np.minimum(np.abs(x), E4M3_MAX)              # satfinite
     _, ex = np.frexp(a)                              # a = f * 2^ex, f in [0.5, 1)
-    k = ex.astype(np.int64) - 1                      # a in [2^k, 2^(k+1))
-    k = np.maximum(k, -6)                            # subnormal range shares 2^-9
-    q = np.ldexp(1.0, k - 3)
-    n = np.rint(a / q)                               # exact scaling, RNE
-    v = n * q
-    v = np.minimum(v, E4M3_MAX)
-    # value -> code: exponent field and mantissa from the value
-    code = np.zeros(a.shape, dtype=np.int64)
-    nz = v > 0
-    _, ev = np.frexp(v[nz])
-    kv = ev.astype(np.int64) - 1
-    sub = kv < -6
-    kv_n = np.where(sub, -6, kv)
-    mant = np.rint(v[nz] / np.ldexp(1.0, kv_n - 3)).astype(np.int64)
-    # normals: mant in [8, 16) -> field e = kv + 7, m = mant - 8
-    # subnormals: mant in [1, 8)  -> field e = 0,   m = mant
-    efield = np.where(sub, 0, kv_n + 7)
-    mfield = np.where(sub, mant, mant - 8)
-    code[nz] = (efield << 3) | mfield
-    code = code | (neg.astype(np.int64) << 7)
+    k = np.maximum(ex - 1, -6)                       # binade; the subnormals share 2^-9
+    n = np.rint(np.ldexp(a, 3 - k))                  # a / 2^(k-3), exact scaling, RNE
+    carry = n >= 16.0
+    k = np.where(carry, k + 1, k)
+    n = np.where(carry, 8.0, n).astype(np.int64)
+    sub = n < 8                                      # only when k == -6
+    efield = np.where(sub, 0, k + 7).astype(np.int64)
+    mfield = np.where(sub, n, n - 8)
+    code = (efield << 3) | mfield | (neg.astype(np.int64) << 7)
     return code.astype(np.uint8)
 
 

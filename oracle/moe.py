@@ -234,7 +234,7 @@ def bias_update(b, counts, T: int, K: int, gamma: float = GAMMA):
 # Whole layer
 # --------------------------------------------------------------------------
 
-def moe_forward(u, e, b, K: int, weights, tokens=None) -> dict:
+def moe_forward(u, e, b, K: int, weights, tokens=None, select=None) -> dict:
     """The layer's forward pass.
 
     u [T, d], e [N_r, d] (bf16 values), b [N_r] (FP32 values).
@@ -242,11 +242,18 @@ def moe_forward(u, e, b, K: int, weights, tokens=None) -> dict:
     tokens: optional 1-D array of token indices; routing, permutation and
     the bias update always cover all T tokens, the expert outputs and the
     combine only the listed tokens (tokens are independent given routing).
+    select: optional [T, K] expert choice to use instead of the oracle's own
+    top-K (to evaluate a token under another, equally valid, selection when
+    two keys are closer than the comparison can resolve); gates are still the
+    oracle's affinities normalised over that selection.
     """
     u = np.asarray(u, np.float64)
     T, d = u.shape
     N_r = e.shape[0]
     s, s32, idx, gates = route(u, e, b, K)
+    if select is not None:
+        idx = np.asarray(select, np.int64)
+        gates = gates_from(s, idx)
     counts, offsets, sorted_token, inv = permute(idx, N_r)
     b_new, ratio = bias_update(b, counts, T, K)
 

@@ -1,0 +1,287 @@
+"""Kernel-by-kernel parity of the CUDA path (through the C ABI) with the CPU
+oracle, on seeded inputs that span several tiles and ragged tails.
+
+Exactness rules: FP8 codes and scales of the quantisers, top-K from given
+scores, the permutation, and the bias update are bit-exact; floating-point
+outputs meet |gpu - ref| <= 8e-3 |ref| + 1e-3 rms(ref).
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import moe as O
+from oracle.e4m3 import round_fp32
+
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL_RMS = 8e-3, 1e-3
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def assert_close(gpu, ref, what):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    err = np.abs(gpu - ref)
+    bound = RTOL * np.abs(ref) + ATOL_RMS * rms
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
+                             f"worst at {i}: gpu={gpu[i]} ref={ref[i]} rms={rms}")
+
+
+# ---------------------------------------------------------------- quantisers
+
+def _activation_rows(rows, cols, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(rows, cols, generator=g)
+    x *= torch.exp2(torch.randint(-30, 30, (rows, 1), generator=g).float())
+    if rows >= 4 and cols >= 256:
+        x[0, :128] = 0.0                         # all-zero tile
+        x[1, 128:256] = -0.0                     # negative zeros
+        x[2, :128] = torch.randn(128, generator=g) * 2.0 ** -130   # bf16 subnormals
+        x[3, :128] = 448.0 * torch.sign(torch.randn(128, generator=g))
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (37, 256), (300, 2048), (1000, 7168)])
+def test_quant_1x128_bit_exact(lib, rows, cols):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    x = _activation_rows(rows, cols, seed=rows)
+    xd = x.cuda()
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows, cols // 128, dtype=torch.float32, device="cuda")
+    B.moe_quant_1x128(xd, q, s)
+    torch.cuda.synchronize()
+    rq, rs = O.quant_1x128(x.double().numpy())
+    assert np.array_equal(s.cpu().double().numpy(), rs)
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (256, 384), (2048, 7168)])
+def test_quant_128x128_bit_exact(lib, rows, cols):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    g = torch.Generator().manual_seed(cols)
+    w = torch.randn(rows, cols, generator=g) * 0.02
+    w[:128, :128] = 0.0
+    if cols >= 256:
+        w[:128, 128:256] *= 1e5
+    wd = w.cuda()
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows // 128, cols // 128, dtype=torch.float32, device="cuda")
+    B.moe_quant_128x128(wd, q, s)
+    torch.cuda.synchronize()
+    rq, rs = O.quant_128x128(w.double().numpy())
+    assert np.array_equal(s.cpu().double().numpy(), rs)
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+# ---------------------------------------------------------------- router
+
+@pytest.mark.parametrize("T,N,K,ties", [(1000, 8, 2, False), (1000, 64, 6, False),
+                                        (777, 256, 8, False), (500, 256, 8, True),
+                                        (300, 64, 16, False), (64, 16, 16, True)])
+def test_topk_from_scores_bit_exact(lib, T, N, K, ties):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    s = workloads.scores(T, N, seed=T + N, ties=ties)
+    b = torch.zeros(N) if ties else (torch.rand(N, generator=torch.Generator().manual_seed(N)) - 0.5) * 0.02
+    idx = torch.empty(T, K, dtype=torch.int32, device="cuda")
+    gates = torch.empty(T, K, dtype=torch.float32, device="cuda")
+    B.moe_route(None, None, b.cuda(), K, idx, gates, scores_in=s.cuda())
+    torch.cuda.synchronize()
+    ref = O.select_topk(s.double().numpy(), b.double().numpy(), K)
+    assert np.array_equal(idx.cpu().numpy(), ref)
+    rg = O.gates_from(s.double().numpy(), ref)
+    assert np.allclose(gates.cpu().double().numpy(), rg, rtol=2e-6, atol=0)
+
+
+def _check_routing(gpu_idx, s64, b, K, margin=1e-5):
+    """Selections equal, except tokens whose K-th and (K+1)-th oracle keys are
+    closer than `margin`. Returns the tokens that differ."""
+    key = s64 + b[None, :]
+    ref = np.argsort(-round_fp32(key), axis=1, kind="stable")
+    diff = []
+    for t in range(gpu_idx.shape[0]):
+        if set(gpu_idx[t]) != set(ref[t, :K]):
+            srt = np.sort(key[t])[::-1]
+            m = srt[K - 1] - srt[K] if K < key.shape[1] else np.inf
+            assert m < margin, f"token {t}: selection differs with margin {m}"
+            diff.append(t)
+    return diff
+
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", None), ("mid", 1000), ("prefill", 1500),
+                                    ("decode", None)])
+def test_router_tensor_cores(lib, name, T):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    cfg = workloads.CONFIGS[name]
+    if T is not None:
+        cfg = cfg.with_tokens(T)
+    u, e, b = workloads.activations(cfg), workloads.centroids(cfg), workloads.bias(cfg)
+    idx = torch.empty(cfg.T, cfg.K_r, dtype=torch.int32, device="cuda")
+    gates = torch.empty(cfg.T, cfg.K_r, dtype=torch.float32, device="cuda")
+    sc = torch.empty(cfg.T, cfg.N_r, dtype=torch.float32, device="cuda")
+    B.moe_route(u.cuda(), e.cuda(), b.cuda(), cfg.K_r, idx, gates, scores_out=sc)
+    torch.cuda.synchronize()
+    s64 = O.router_scores(u.double().numpy(), e.double().numpy())
+    assert np.abs(sc.cpu().double().numpy() - s64).max() < 1e-5
+    gi = idx.cpu().numpy()
+    diff = _check_routing(gi, s64, b.double().numpy(), cfg.K_r)
+    assert len(diff) <= max(2, cfg.T // 200)
+    rg = O.gates_from(s64, gi.astype(np.int64))
+    assert np.allclose(gates.cpu().double().numpy(), rg, rtol=1e-4, atol=1e-6)
+
+
+# ---------------------------------------------------------------- permutation
+
+@pytest.mark.parametrize("T,N,K,pattern", [(1, 8, 2, "uniform"), (255, 8, 2, "uniform"),
+                                           (257, 256, 8, "uniform"), (5000, 64, 6, "uniform"),
+                                           (3000, 256, 8, "one_hot_expert"), (600, 1024, 16, "uniform"),
+                                           (1000, 16, 16, "first_k"), (100, 4, 1, "uniform")])
+def test_permute_bit_exact(lib, T, N, K, pattern):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    idx = workloads.topk_indices(T, N, K, seed=T * 7 + N, pattern=pattern)
+    d = 256
+    g = torch.Generator().manual_seed(T)
+    xq = torch.randint(0, 256, (T, d), generator=g, dtype=torch.uint8)
+    xs = torch.rand(T, d // 128, generator=g)
+    dev = dict(device="cuda")
+    counts = torch.empty(N, dtype=torch.int32, **dev)
+    offsets = torch.empty(N + 1, dtype=torch.int32, **dev)
+    st = torch.empty(T * K, dtype=torch.int32, **dev)
+    inv = torch.empty(T, K, dtype=torch.int32, **dev)
+    xqp = torch.empty(T * K, d, dtype=torch.uint8, **dev)
+    xsp = torch.empty(T * K, d // 128, dtype=torch.float32, **dev)
+    ws = torch.empty(max(B.moe_permute_workspace(T, N), 16), dtype=torch.uint8, **dev)
+    B.moe_permute(idx.cuda(), N, counts, offsets, st, inv, ws, xq.cuda(), xs.cuda(), xqp, xsp)
+    torch.cuda.synchronize()
+    rc, ro, rst, rinv = O.permute(idx.numpy(), N)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(st.cpu().numpy(), rst)
+    assert np.array_equal(inv.cpu().numpy(), rinv)
+    assert np.array_equal(xqp.cpu().numpy(), xq.numpy()[rst])
+    assert np.array_equal(xsp.cpu().numpy(), xs.numpy()[rst])
+
+
+# ---------------------------------------------------------------- combine, bias
+
+@pytest.mark.parametrize("T,K,d", [(1, 1, 8), (333, 2, 256), (1000, 8, 7168)])
+def test_combine(lib, T, K, d):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    g = torch.Generator().manual_seed(T + d)
+    u = torch.randn(T, d, generator=g).to(torch.bfloat16)
+    ysh = (torch.randn(T, d, generator=g) * 0.1).to(torch.bfloat16)
+    yp = (torch.randn(T * K, d, generator=g) * 0.1).to(torch.bfloat16)
+    inv = torch.randperm(T * K, generator=g).reshape(T, K).to(torch.int32)
+    gt = torch.rand(T, K, generator=g)
+    gt = gt / gt.sum(dim=1, keepdim=True)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    B.moe_combine(u.cuda(), yp.cuda(), ysh.cuda(), inv.cuda(), gt.cuda(), out)
+    torch.cuda.synchronize()
+    ref = O.combine(u.double().numpy(), yp.double().numpy(), ysh.double().numpy(),
+                    inv.numpy(), gt.double().numpy())
+    assert_close(f64(out), ref, "combine")
+
+
+@pytest.mark.parametrize("N,T,K", [(8, 64, 2), (256, 8192, 8), (64, 4095, 6), (256, 0, 8)])
+def test_bias_update_bit_exact(lib, N, T, K):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    g = torch.Generator().manual_seed(N + T)
+    b = (torch.rand(N, generator=g) - 0.5) * 0.02
+    if T:
+        idx = workloads.topk_indices(T, N, K, seed=N)
+        counts = torch.bincount(idx.reshape(-1).long(), minlength=N).to(torch.int32)
+        counts[0] = (T * K) // N if (T * K) % N == 0 else counts[0]
+    else:
+        counts = torch.zeros(N, dtype=torch.int32)
+    bd = b.cuda()
+    mom = torch.zeros(1, device="cuda")
+    B.moe_bias_update(bd, counts.cuda(), T, K, 0.001, mom)
+    torch.cuda.synchronize()
+    rb, ratio = O.bias_update(b.double().numpy(), counts.numpy(), T, K)
+    assert np.array_equal(bd.cpu().double().numpy(), rb)
+    assert abs(mom.item() - ratio) <= 1e-6 * max(ratio, 1.0)
+
+
+# ---------------------------------------------------------------- grouped GEMM
+
+def _gemm_case(d, I, counts, T, seed):
+    """Oracle-quantised inputs for the grouped GEMM alone."""
+    rng = np.random.default_rng(seed)
+    N_r = len(counts)
+    P = int(sum(counts))
+    xp = round_fp32(rng.standard_normal((P, d)) * np.exp2(rng.integers(-3, 3, (P, 1))))
+    xsh = round_fp32(rng.standard_normal((T, d)))
+    xq_p, xs_p = O.quant_1x128(xp)
+    xq, xs = O.quant_1x128(xsh)
+    experts = []
+    for _ in range(N_r + 1):
+        w = [round_fp32(rng.standard_normal(sh) * 0.02) for sh in [(I, d), (I, d), (d, I)]]
+        experts.append(O.quantise_expert(*w))
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    return xq_p, xs_p, xq, xs, experts, offsets
+
+
+@pytest.mark.parametrize("d,I,counts,T", [
+    (256, 128, [0, 1, 130, 257], 100),
+    (512, 256, [3, 0, 128, 64, 200], 129),
+    (2048, 1024, [384, 200], 256),
+    (7168, 2048, [5, 300], 130),
+])
+def test_grouped_gemm_fp8(lib, d, I, counts, T):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    xq_p, xs_p, xq, xs, experts, offsets = _gemm_case(d, I, counts, T, seed=d + I)
+    N_r = len(counts)
+    P = int(offsets[-1])
+    K_r = P // T if P % T == 0 else None
+    # the C ABI sizes y_perm as T*K_r rows; pad the routed rows to that
+    K_r = -(-P // T)
+    Ppad = T * K_r
+    dev = dict(device="cuda")
+    cu = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
+    xq_pd = torch.zeros(Ppad, d, dtype=torch.uint8, **dev)
+    xs_pd = torch.ones(Ppad, d // 128, dtype=torch.float32, **dev)
+    xq_pd[:P] = cu(xq_p, torch.uint8)
+    xs_pd[:P] = cu(xs_p, torch.float32)
+    stack = lambda key, dt: cu(np.stack([e[key] for e in experts]), dt)
+    wg, wu, wd = stack("gate_q", torch.uint8), stack("up_q", torch.uint8), stack("down_q", torch.uint8)
+    sg, su, sd = stack("gate_s", torch.float32), stack("up_s", torch.float32), stack("down_s", torch.float32)
+    off = torch.from_numpy(offsets).cuda()
+    y_perm = torch.empty(Ppad, d, dtype=torch.bfloat16, **dev)
+    y_sh = torch.empty(T, d, dtype=torch.bfloat16, **dev)
+    ws = torch.empty(B.moe_grouped_gemm_fp8_workspace(T, K_r, d, I), dtype=torch.uint8, **dev)
+    B.moe_grouped_gemm_fp8(xq_pd, xs_pd, off, cu(xq, torch.uint8), cu(xs, torch.float32),
+                           wg, wu, wd, sg, su, sd, y_perm, y_sh, ws)
+    torch.cuda.synchronize()
+    assert B.moe_get_error() == 0
+    yp = f64(y_perm)
+    for i in range(N_r):
+        a, b_ = offsets[i], offsets[i + 1]
+        if b_ > a:
+            ref, _ = O.expert_ffn(xq_p[a:b_], xs_p[a:b_], experts[i])
+            assert_close(yp[a:b_], ref, f"expert {i}")
+    ref, _ = O.expert_ffn(xq, xs, experts[N_r])
+    assert_close(f64(y_sh), ref, "shared expert")
+
+
+# ---------------------------------------------------------------- failure path
+
+def test_wait_timeout_sets_error_word(lib):
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    assert B.moe_get_error() == 0
+    B.moe_debug_wait_timeout(2000)           # a 2 ms wait on a barrier nothing signals
+    assert B.moe_get_error() == 4            # MOE_ERR_TIMEOUT, read and cleared
+    assert B.moe_get_error() == 0
+    x = torch.zeros(4, 128, dtype=torch.bfloat16, device="cuda")   # the context still works
+    q = torch.empty(4, 128, dtype=torch.uint8, device="cuda")
+    s = torch.empty(4, 1, dtype=torch.float32, device="cuda")
+    B.moe_quant_1x128(x, q, s)
+    torch.cuda.synchronize()
+    assert s.cpu().eq(1.0).all()

@@ -1,0 +1,112 @@
+"""End-to-end parity of the whole layer (MoELayerFP8 over the C ABI) with
+the CPU oracle on the five workloads.
+
+tiny and mid are compared on every token. prefill, decode and skew run at
+full size in the same launch configuration as the benchmark; the oracle
+routes all tokens (selection, counts, bias update) and computes the expert
+outputs for a seeded sample of tokens. Weights are drawn on the device by the
+seeded generator; the oracle receives the same FP32 weights copied to the
+host and quantises them itself (its codes and scales must equal the GPU's).
+"""
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import moe as O
+from tests.test_gpu_kernels import _check_routing, assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _build(cfg, weights_on="cuda"):
+    from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
+    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I)
+    for slot in range(cfg.N_r + 1):
+        w = workloads.expert_weights(cfg, slot, device=weights_on)
+        layer.load_expert(slot, *[x.cuda() for x in w])
+    return layer
+
+
+def _run(cfg, sample, weights_on):
+    dev_inputs = cfg.T * cfg.d > 8_000_000
+    gen_dev = "cuda" if dev_inputs else "cpu"
+    u = workloads.activations(cfg, device=gen_dev)
+    e = workloads.centroids(cfg, device=gen_dev)
+    b = workloads.bias(cfg, device=gen_dev)
+    layer = _build(cfg, weights_on)
+    ud, ed, bd = u.cuda(), e.cuda(), b.cuda().clone()
+    out = layer.forward(ud, ed, bd, update_bias=True)
+    torch.cuda.synchronize()
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    assert B.moe_get_error() == 0
+
+    un, en, bn = u.cpu().double().numpy(), e.cpu().double().numpy(), b.cpu().double().numpy()
+    gpu_idx = layer.topk_idx.cpu().numpy().astype(np.int64)
+    s64 = O.router_scores(un, en)
+    diff = _check_routing(gpu_idx, s64, bn, cfg.K_r)
+    assert len(diff) <= max(2, cfg.T // 200), len(diff)
+
+    # permutation and bias update given the GPU's selection: bit-exact
+    rc, ro, rst, rinv = O.permute(gpu_idx, cfg.N_r)
+    assert np.array_equal(layer.counts.cpu().numpy(), rc)
+    assert np.array_equal(layer.offsets.cpu().numpy(), ro)
+    assert np.array_equal(layer.sorted_token.cpu().numpy(), rst)
+    assert np.array_equal(layer.inv.cpu().numpy(), rinv)
+    rb, ratio = O.bias_update(bn, rc, cfg.T, cfg.K_r)
+    assert np.array_equal(bd.cpu().double().numpy(), rb)
+
+    # expert outputs and h' on the sample, under the GPU's selection; the
+    # oracle quantises the same FP32 weights itself (threads: numpy releases
+    # the GIL), and its codes and scales must equal the GPU's
+    slots = sorted(set(gpu_idx[sample].reshape(-1).tolist()) | {cfg.N_r})
+    host_w = {s_: [x.cpu().double().numpy() for x in workloads.expert_weights(cfg, s_, device=weights_on)]
+              for s_ in slots}
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        quant = dict(zip(slots, ex.map(lambda s_: O.quantise_expert(*host_w[s_]), slots)))
+    del host_w
+    for s_, q in quant.items():
+        for key, t in [("gate_q", layer.w_gate), ("up_q", layer.w_up), ("down_q", layer.w_down)]:
+            assert np.array_equal(t[s_].cpu().numpy(), q[key]), (s_, key)
+        for key, t in [("gate_s", layer.s_gate), ("up_s", layer.s_up), ("down_s", layer.s_down)]:
+            assert np.array_equal(t[s_].cpu().double().numpy(), q[key]), (s_, key)
+    weights = quant.__getitem__
+
+    ref = O.moe_forward(un, en, bn, cfg.K_r, weights, tokens=sample, select=gpu_idx)
+    assert np.array_equal(layer.xq[torch.as_tensor(sample).cuda()].cpu().numpy(), ref["xq"])
+    assert_close(f64(layer.y_shared)[sample], ref["y_shared"], "shared expert")
+    yp = f64(layer.y_perm)
+    inv = layer.inv.cpu().numpy()
+    for j, t in enumerate(sample):
+        assert_close(yp[inv[t]], ref["y_routed"][j], f"routed rows of token {t}")
+    assert_close(f64(out)[sample], ref["out"], "h'")
+    return layer
+
+
+def _sample(cfg, n, seed):
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(1, cfg.T - 1), size=min(n, cfg.T - 2), replace=False)
+    return np.unique(np.concatenate([[0, cfg.T - 1], mid]))
+
+
+def test_layer_tiny_all_tokens(lib):
+    cfg = workloads.CONFIGS["tiny"]
+    _run(cfg, np.arange(cfg.T), weights_on="cpu")
+
+
+def test_layer_tiny_ragged_tokens(lib):
+    cfg = workloads.CONFIGS["tiny"].with_tokens(37)
+    _run(cfg, np.arange(cfg.T), weights_on="cpu")
+
+
+def test_layer_mid_sampled(lib):
+    cfg = workloads.CONFIGS["mid"]
+    _run(cfg, _sample(cfg, 62, seed=1), weights_on="cuda")
+
+
+@pytest.mark.parametrize("name,n", [("decode", 6), ("prefill", 4), ("skew", 4)])
+def test_layer_full_size_sampled(lib, name, n):
+    cfg = workloads.CONFIGS[name]
+    _run(cfg, _sample(cfg, n, seed=3), weights_on="cuda")
