@@ -22,6 +22,7 @@ _z = ctypes.c_size_t
 SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
     "moe_version": (_i, []),
+    "moe_last_error_detail": (ctypes.c_char_p, []),
     "moe_get_error": (_i, [ctypes.POINTER(_i)]),
     "moe_quant_1x128": (_i, [_p, _i, _i, _p, _p, _p]),
     "moe_quant_128x128": (_i, [_p, _i, _i, _p, _p, _p]),
@@ -50,7 +51,8 @@ _lib = None
 class MoEError(RuntimeError):
     def __init__(self, call: str, status: int):
         self.status = status
-        super().__init__(f"{call} failed: {status_string(status)} ({status})")
+        detail = load().moe_last_error_detail().decode(errors="replace")
+        super().__init__(f"{call} failed: {status_string(status)} ({status}) [{detail}]")
 
 
 def load() -> ctypes.CDLL:

@@ -144,11 +144,13 @@ extern "C" int moe_debug_wait_timeout(int timeout_us, void* stream) {
 extern "C" int moe_get_error(int* device_status) {
   using namespace moe;
   MOE_CHECK_ARG(device_status);
-  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (int st = cuda_status(cudaDeviceSynchronize(), "moe_get_error: synchronize")) return st;
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (int st = cuda_status(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)), "moe_get_error: read"))
+    return st;
   const int zero = 0;
-  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (int st = cuda_status(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)), "moe_get_error: clear"))
+    return st;
   *device_status = v;
   return MOE_OK;
 }
@@ -166,3 +168,5 @@ extern "C" const char* moe_status_string(int status) {
 }
 
 extern "C" int moe_version(void) { return 100; }
+
+extern "C" const char* moe_last_error_detail(void) { return moe::last_error_buf(); }

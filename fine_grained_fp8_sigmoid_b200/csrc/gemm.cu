@@ -14,12 +14,15 @@
 // TMEM plays that role with two partial buffers in flight, so the next block's
 // MMAs overlap the FMAs of the current one.
 //
-// Structure (one persistent CTA per SM, 320 threads):
-//   warp 0    TMA producer: A tile 128 x 128 and B tile 256 x 128 per K block
-//             (128-byte swizzle), 4-stage ring.
-//   warp 1    MMA issuer (one thread) and TMEM owner (512 columns = 2 x 256).
-//   warps 2-9 epilogue: warp w reads TMEM lanes 32*(w%4).. (rows), and
-//             (w-2)/4 selects the column half.
+// Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
+//   warp 0     TMA producer: A tile 128 x 128 and B tile 256 x 128 per K block
+//              (128-byte swizzle), 4-stage ring.
+//   warp 1     MMA issuer (one thread) and TMEM owner (512 columns = 2 x 256).
+//   warps 2-3  idle (they complete the first warpgroup).
+//   warps 4-11 epilogue: warp w reads TMEM lanes 32*(w%4).. (rows), and
+//              (w-4)/4 selects the column half. Each thread keeps 128 FP32
+//              accumulators, so the epilogue warpgroups take 224 registers
+//              per thread and the first warpgroup gives its share back (56).
 //
 // Two launches:
 //   phase 1: per tile (group g, 128 rows, 128 intermediate channels n):
@@ -43,8 +46,13 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 320;
+constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
+constexpr int EPI_WARP0 = 4;     // first epilogue warp
+// launch at 168 registers (65536 / 384, rounded down to 8); then
+// 128 * 56 + 256 * 224 = 384 * 168, and 56 + 2 * 224 <= 512 per sub-partition
+constexpr uint32_t REGS_CTRL = 56;
+constexpr uint32_t REGS_EPI = 224;
 constexpr int MAX_GROUPS = 1025;
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -115,7 +123,7 @@ __device__ __forceinline__ Tile decode_tile(const Smem& sm, const Args& a, int t
 __device__ __forceinline__ float silu(float x) { return __fdiv_rn(x, 1.0f + expf(-x)); }
 
 template <int PHASE>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                         const Args a) {
@@ -186,6 +194,7 @@ __global__ void __maxnreg__(200)
   const uint32_t tmem = sm.tmem_base;
   const int total = sm.total_tiles;
   volatile int* abort = &sm.abort;
+  if (warp < EPI_WARP0) regs_decrease<REGS_CTRL>();
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
@@ -259,10 +268,11 @@ __global__ void __maxnreg__(200)
       volatile int never = 0;
       mbar_wait(&sm.drain, 0, &never, 100000000ull);
     }
-  } else {
+  } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------ epilogue
+    regs_increase<REGS_EPI>();
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;
+    const int half = (warp - EPI_WARP0) >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int buf = 0;
@@ -416,7 +426,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   using namespace moe;
   using namespace moe::gg;
   MOE_CHECK_ARG(N_r >= 1 && K_r >= 1 && T >= 0 && d > 0 && I > 0);
-  MOE_CHECK_SUPPORTED(N_r + 1 <= MAX_GROUPS && K_r <= N_r && d % 256 == 0 && I % 128 == 0);
+  MOE_CHECK_SUPPORTED(N_r + 1 <= MAX_GROUPS && d % 256 == 0 && I % 128 == 0);
   const long long P = static_cast<long long>(T) * K_r;
   MOE_CHECK_SUPPORTED(P + T < (1LL << 31) && static_cast<long long>(N_r + 1) * (d > I ? d : I) < (1LL << 31));
   if (T == 0) return MOE_OK;
@@ -467,11 +477,14 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
 
   auto k1 = grouped_gemm_kernel<1>;
   auto k2 = grouped_gemm_kernel<2>;
-  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)) != cudaSuccess ||
-      cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  if (int st = cuda_status(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(SMEM_BYTES)), "smem attribute (gate/up)"))
+    return st;
+  if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(SMEM_BYTES)), "smem attribute (down)"))
+    return st;
   k1<<<g1, THREADS, SMEM_BYTES, s>>>(tmA, tmX, tmWg, tmWu, args);
-  if (int st = launch_status()) return st;
+  if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
   k2<<<g2, THREADS, SMEM_BYTES, s>>>(tmH, tmH, tmWd, tmWd, args);
-  return launch_status();
+  return launch_status("grouped GEMM launch (down)");
 }

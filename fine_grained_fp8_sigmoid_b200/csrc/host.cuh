@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cudaTypedefs.h>
+#include <cstdio>
 #include <mutex>
 
 #include "common.cuh"
@@ -18,9 +19,24 @@ namespace moe {
     if (!(cond)) return MOE_ERR_UNSUPPORTED; \
   } while (0)
 
-inline int launch_status() {
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+// Text of the last host-side failure in this thread (moe_last_error_detail).
+inline char* last_error_buf() {
+  static thread_local char buf[256] = {0};
+  return buf;
+}
+
+inline int record_failure(int status, const char* where, const char* what) {
+  snprintf(last_error_buf(), 256, "%s: %s", where, what);
+  return status;
+}
+
+inline int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MOE_OK;
+  return record_failure(MOE_ERR_CUDA, where, cudaGetErrorString(e));
+}
+
+inline int launch_status(const char* where = "kernel launch") {
+  return cuda_status(cudaGetLastError(), where);
 }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -72,7 +88,7 @@ inline int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
                         int elem_bytes, uint64_t rows, uint64_t cols, uint32_t box_rows,
                         uint32_t box_cols) {
   auto enc = tensor_map_encoder();
-  if (!enc) return MOE_ERR_CUDA;
+  if (!enc) return record_failure(MOE_ERR_CUDA, "cuTensorMapEncodeTiled", "entry point not found");
   if (reinterpret_cast<uintptr_t>(base) % 16 != 0) return MOE_ERR_INVALID_ARG;
   if ((cols * elem_bytes) % 16 != 0) return MOE_ERR_UNSUPPORTED;
   cuuint64_t dims[2] = {cols, rows};
@@ -82,7 +98,14 @@ inline int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
   CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+  if (r != CUDA_SUCCESS) {
+    char what[96];
+    snprintf(what, sizeof what, "CUresult %d (rows %llu, cols %llu, box %ux%u)", static_cast<int>(r),
+             static_cast<unsigned long long>(rows), static_cast<unsigned long long>(cols), box_rows,
+             box_cols);
+    return record_failure(MOE_ERR_CUDA, "cuTensorMapEncodeTiled", what);
+  }
+  return MOE_OK;
 }
 
 }  // namespace moe

@@ -2,12 +2,18 @@
 // gates ("DeepSeek-V3 Teknik Raporu", Yöntem 2; "DeepSeek-V3 Technical
 // Report" (fr), Méthode 2).
 //
-// The logits are a [T x d] x [d x N_r] product: one CTA takes 128 tokens and
-// all N_r experts, streams u and e through shared memory with TMA (128-byte
-// swizzled K blocks of 64 bf16), and accumulates u . e^T in TMEM with
-// tcgen05 kind::f16 MMAs (BF16 inputs, FP32 accumulation). Four epilogue
-// warps then own one token row each (one TMEM lane) and do sigmoid, the
-// biased top-K and the gates in registers.
+// The logits are a [T x d] x [d x N_r] product on the tensor cores. One CTA
+// takes 128 tokens and all experts (the MMA is N = 256; experts beyond N_r
+// read zero rows). u and e stream through shared memory with TMA in 128-byte
+// swizzled K blocks of 64 bf16. Each K block's four tcgen05 kind::f16 MMAs
+// (BF16 x BF16 -> FP32) write a fresh TMEM partial, and the epilogue warps add
+// the partials in FP32 registers. Accumulating all of d = 7168 inside the
+// tensor core lets its truncating accumulation drift by ~1e-4 in the logit;
+// summing 64-wide partials in registers keeps the error near FP32 rounding,
+// the same promotion the FP8 GEMMs use.
+// Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
+// epilogue (TMEM lane quadrant w%4, column half (w-4)/4), which finishes
+// with sigmoid, the biased top-K of each half, and a merge of the halves.
 #include "host.cuh"
 
 namespace moe {
@@ -15,14 +21,18 @@ namespace route {
 
 constexpr int BM = 128;          // tokens per CTA (TMEM lanes)
 constexpr int BK = 64;           // bf16 per K block = 128 bytes = one swizzle row
+constexpr int NP = 256;          // MMA N: all experts of a token in one tile
 constexpr int STAGES = 4;
-constexpr int THREADS = 192;     // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int THREADS = 384;
+constexpr int EPI_WARP0 = 4;
+constexpr int EPI_THREADS = 256;
 constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = NP * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * NP;
+constexpr uint32_t REGS_CTRL = 56;
+constexpr uint32_t REGS_EPI = 224;
 
-// Inserts (key, idx, s) into a list sorted by key descending; candidates
-// arrive in increasing idx, so a candidate never passes an equal key (equal
-// keys keep the lower index first). Once a slot is taken, the rest of the
-// list shifts down by one.
 template <int KMAX>
 __device__ __forceinline__ void topk_insert(float (&kk)[KMAX], int (&ii)[KMAX], float (&ss)[KMAX],
                                             float key, int idx, float s) {
@@ -74,28 +84,37 @@ __device__ __forceinline__ void topk_store(const int (&ii)[KMAX], const float (&
 
 __device__ __forceinline__ float sigmoidf(float z) { return __fdiv_rn(1.0f, 1.0f + expf(-z)); }
 
+template <int KMAX>
 struct Smem {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
-  uint64_t acc_full;
+  uint64_t tfull[2];
+  uint64_t tempty[2];
   uint64_t drain;
+  uint64_t xbar;
   uint32_t tmem_base;
   int abort;
-  float bias[256];
+  float bias[NP];
+  float m_key[KMAX][BM];   // top-K of the upper column half, handed to the lower half
+  int m_idx[KMAX][BM];
+  float m_s[KMAX][BM];
 };
+
+template <int KMAX>
+constexpr size_t router_smem_bytes() {
+  return 1024 + STAGES * STAGE_BYTES + sizeof(Smem<KMAX>);
+}
 
 template <int KMAX>
 __global__ void __launch_bounds__(THREADS, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_e,
-                  const float* __restrict__ b, int T, int d, int N_r, int NP, int K,
+                  const float* __restrict__ b, int T, int d, int N_r, int K,
                   float* __restrict__ scores_out, int32_t* __restrict__ topk_idx,
-                  float* __restrict__ gates, uint32_t tmem_cols) {
+                  float* __restrict__ gates) {
   extern __shared__ uint8_t smem_raw[];
   // operand tiles need 1024-byte alignment for the 128-byte swizzle
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int b_bytes = NP * BK * 2;
-  const int stage_bytes = A_BYTES + b_bytes;
-  Smem& sm = *reinterpret_cast<Smem*>(tiles + STAGES * stage_bytes);
+  Smem<KMAX>& sm = *reinterpret_cast<Smem<KMAX>*>(tiles + STAGES * STAGE_BYTES);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
@@ -107,8 +126,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    mbar_init(&sm.acc_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], EPI_THREADS / 32);
+    }
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.xbar, EPI_THREADS);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -117,102 +140,142 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tm_e);
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, tmem_cols);
+    tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < N_r; i += THREADS) sm.bias[i] = b[i];
+  for (int i = threadIdx.x; i < NP; i += THREADS) sm.bias[i] = i < N_r ? b[i] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // producer: K blocks of u (128 x 64) and e (NP x 64)
-      int armed_parity[STAGES];
-      for (int s = 0; s < STAGES; ++s) armed_parity[s] = -1;
+  if (warp < EPI_WARP0) {
+    regs_decrease<REGS_CTRL>();
+    if (warp == 0 && lane == 0) {
+      // producer: K blocks of u (128 x 64) and e (256 x 64, rows >= N_r read as zero)
+      int armed[STAGES];
+      for (int s = 0; s < STAGES; ++s) armed[s] = -1;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (kb / STAGES) & 1;
         if (!mbar_wait(&sm.empty[s], ph ^ 1, abort)) break;
-        uint8_t* a_dst = tiles + s * stage_bytes;
-        mbar_arrive_expect_tx(&sm.full[s], stage_bytes);
+        uint8_t* a_dst = tiles + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&sm.full[s], STAGE_BYTES);
         tma_load_2d(a_dst, &tm_u, &sm.full[s], kb * BK, tile * BM);
         tma_load_2d(a_dst + A_BYTES, &tm_e, &sm.full[s], kb * BK, 0);
-        armed_parity[s] = ph;
+        armed[s] = ph;
       }
       if (*abort) {
         // let every issued copy land before the block's shared memory is released
         volatile int never = 0;
         for (int s = 0; s < STAGES; ++s)
-          if (armed_parity[s] >= 0) mbar_wait(&sm.full[s], armed_parity[s], &never, 100000000ull);
+          if (armed[s] >= 0) mbar_wait(&sm.full[s], armed[s], &never, 100000000ull);
       }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
       const uint32_t idesc = make_idesc(1, 1, BM, NP);
+      int buf = 0;
+      uint32_t tphase = 0;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (kb / STAGES) & 1;
+        if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) break;
         if (!mbar_wait(&sm.full[s], ph, abort)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(tiles + s * stage_bytes);
+        const uint32_t a_addr = smem_u32(tiles + s * STAGE_BYTES);
         const uint64_t ad = sw128_kmajor_desc(a_addr);
         const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes per MMA
-          umma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+          umma_f16(tmem + buf * NP, ad + 2 * k, bd + 2 * k, idesc, k != 0);
         umma_commit(&sm.empty[s]);
+        umma_commit(&sm.tfull[buf]);
+        buf ^= 1;
+        if (buf == 0) tphase ^= 1;
       }
-      umma_commit(&sm.acc_full);
       // all MMAs of this thread complete before TMEM is released
       umma_commit(&sm.drain);
       volatile int never = 0;
       mbar_wait(&sm.drain, 0, &never, 100000000ull);
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31
+    regs_increase<REGS_EPI>();
     const int q = warp & 3;
+    const int half = (warp - EPI_WARP0) >> 2;
     const int r = q * 32 + lane;
     const int t = tile * BM + r;
-    if (warp_wait(&sm.acc_full, 0, abort)) {
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    float acc[128];
+#pragma unroll
+    for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+    int buf = 0;
+    uint32_t tphase = 0;
+    bool ok = true;
+    for (int kb = 0; kb < KB; ++kb) {
+      if (!warp_wait(&sm.tfull[buf], tphase, abort)) { ok = false; break; }
       tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + buf * NP + half * 128 + c * 32, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[c * 32 + j] += v[j];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+      buf ^= 1;
+      if (buf == 0) tphase ^= 1;
+    }
+    if (ok) {
       float kk[KMAX], ss[KMAX];
       int ii[KMAX];
       topk_init(kk, ii, ss);
-      for (int c0 = 0; c0 < NP; c0 += 32) {
-        float v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int col = c0 + j;
-          if (col < N_r) {
-            const float s = sigmoidf(v[j]);
-            v[j] = s;
-            topk_insert(kk, ii, ss, s + sm.bias[col], col, s);
-          }
-        }
-        if (scores_out != nullptr && t < T) {
-          float* dst = scores_out + static_cast<size_t>(t) * N_r + c0;
-          const int ncol = min(32, N_r - c0);
-          if ((N_r & 3) == 0 && ncol == 32) {
+      for (int j = 0; j < 128; ++j) {
+        const int col = half * 128 + j;
+        const float sg = sigmoidf(acc[j]);
+        acc[j] = sg;
+        if (col < N_r) topk_insert(kk, ii, ss, sg + sm.bias[col], col, sg);
+      }
+      if (scores_out != nullptr && t < T) {
+        float* dst = scores_out + static_cast<size_t>(t) * N_r + half * 128;
+        const int ncol = min(128, N_r - half * 128);
+        if ((N_r & 3) == 0 && ncol == 128) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-          } else {
-            for (int j = 0; j < ncol; ++j) dst[j] = v[j];
-          }
+          for (int j = 0; j < 128; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j < ncol) dst[j] = acc[j];
         }
       }
-      if (t < T) topk_store(ii, ss, K, topk_idx + static_cast<size_t>(t) * K, gates + static_cast<size_t>(t) * K);
+      // the upper half hands its list to the lower half, which merges: every
+      // upper-half index exceeds every lower-half one, and the list arrives
+      // in (key desc, index asc) order, so equal keys stay lowest-index first
+      if (half == 1) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          sm.m_key[j][r] = kk[j];
+          sm.m_idx[j][r] = ii[j];
+          sm.m_s[j][r] = ss[j];
+        }
+      }
+      mbar_arrive(&sm.xbar);
+      if (half == 0 && warp_wait(&sm.xbar, 0, abort)) {
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (sm.m_idx[j][r] < N_r) topk_insert(kk, ii, ss, sm.m_key[j][r], sm.m_idx[j][r], sm.m_s[j][r]);
+        if (t < T) topk_store(ii, ss, K, topk_idx + static_cast<size_t>(t) * K, gates + static_cast<size_t>(t) * K);
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -265,22 +328,24 @@ extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
   }
   MOE_CHECK_ARG(u && e && d > 0);
   MOE_CHECK_SUPPORTED(d % BK == 0);
-  const int NP = ((N_r + 15) / 16) * 16;
-  uint32_t tmem_cols = 32;
-  while (static_cast<int>(tmem_cols) < NP) tmem_cols *= 2;
   CUtensorMap tm_u, tm_e;
   if (int st = make_tmap_2d(&tm_u, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, d, BM, BK)) return st;
   if (int st = make_tmap_2d(&tm_e, e, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N_r, d, NP, BK)) return st;
-  const size_t smem = 1024 + STAGES * (A_BYTES + NP * BK * 2) + sizeof(Smem);
   const int blocks = (T + BM - 1) / BM;
   if (K_r <= 8) {
     auto k = router_kernel<8>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, NP, K_r, scores_out, topk_idx, gates, tmem_cols);
+    constexpr size_t smem = router_smem_bytes<8>();
+    if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                             "router smem attribute"))
+      return st;
+    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, K_r, scores_out, topk_idx, gates);
   } else {
     auto k = router_kernel<16>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, NP, K_r, scores_out, topk_idx, gates, tmem_cols);
+    constexpr size_t smem = router_smem_bytes<16>();
+    if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                             "router smem attribute"))
+      return st;
+    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, K_r, scores_out, topk_idx, gates);
   }
   return launch_status();
 }

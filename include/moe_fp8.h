@@ -66,6 +66,13 @@ MOE_API const char* moe_status_string(int status);
 MOE_API int moe_version(void);
 
 /*
+ * Text describing the last host-side failure of a call made by this thread
+ * (which CUDA call failed and its error string). Static per-thread buffer;
+ * empty if nothing has failed.
+ */
+MOE_API const char* moe_last_error_detail(void);
+
+/*
  * moe_get_error: synchronises the device, then reads and clears the device
  * error word that kernels set when a bounded wait gave up.
  *   device_status (HOST pointer, out): MOE_OK or MOE_ERR_TIMEOUT.
