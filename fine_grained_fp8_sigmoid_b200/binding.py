@@ -128,8 +128,8 @@ def moe_grouped_gemm_fp8(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down
     _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
     _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
     _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
-    _want(y_perm, torch.bfloat16, (P, d), "y_perm")
-    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
+    _want(y_perm, torch.float32, (P, d), "y_perm")
+    _want(y_shared, torch.float32, (T, d), "y_shared")
     if T and P != T * K_r:
         raise ValueError("xq_perm rows must be T * K_r")
     check("moe_grouped_gemm_fp8", _lib.load().moe_grouped_gemm_fp8(
@@ -143,8 +143,8 @@ def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
     T, d = u.shape
     K_r = inv.shape[1]
     _want(u, torch.bfloat16, (T, d), "u")
-    _want(y_perm, torch.bfloat16, (T * K_r, d), "y_perm")
-    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
+    _want(y_perm, torch.float32, (T * K_r, d), "y_perm")
+    _want(y_shared, torch.float32, (T, d), "y_shared")
     _want(inv, torch.int32, (T, K_r), "inv")
     _want(gates, torch.float32, (T, K_r), "gates")
     _want(out, torch.bfloat16, (T, d), "out")

@@ -8,8 +8,8 @@ namespace moe {
 // One block per token; each thread handles 8 consecutive channels (16 bytes
 // of bf16) per step. FP32 sum in the fixed order: u, shared, k = 0..K-1.
 __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ u,
-                                                      const uint16_t* __restrict__ y_perm,
-                                                      const uint16_t* __restrict__ y_shared,
+                                                      const float* __restrict__ y_perm,
+                                                      const float* __restrict__ y_shared,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gates, int K,
                                                       int d, int P, uint16_t* out) {
@@ -29,26 +29,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
   const size_t base = static_cast<size_t>(t) * d;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     const uint4 a = *reinterpret_cast<const uint4*>(u + base + c);
-    const uint4 sh = __ldg(reinterpret_cast<const uint4*>(y_shared + base + c));
-    float acc[8];
+    const float4 sh0 = __ldg(reinterpret_cast<const float4*>(y_shared + base + c));
+    const float4 sh1 = __ldg(reinterpret_cast<const float4*>(y_shared + base + c + 4));
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t sw[4] = {sh.x, sh.y, sh.z, sh.w};
+    const float sv[8] = {sh0.x, sh0.y, sh0.z, sh0.w, sh1.x, sh1.y, sh1.z, sh1.w};
+    float acc[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = bf16_bits_to_float(aw[i] & 0xFFFF) + bf16_bits_to_float(sw[i] & 0xFFFF);
-      acc[2 * i + 1] = bf16_bits_to_float(aw[i] >> 16) + bf16_bits_to_float(sw[i] >> 16);
+      acc[2 * i] = bf16_bits_to_float(aw[i] & 0xFFFF) + sv[2 * i];
+      acc[2 * i + 1] = bf16_bits_to_float(aw[i] >> 16) + sv[2 * i + 1];
     }
     for (int k = 0; k < K; ++k) {
       const int r = s_row[k];
       if (r < 0) continue;
       const float g = s_g[k];
-      const uint4 y = __ldg(reinterpret_cast<const uint4*>(y_perm + static_cast<size_t>(r) * d + c));
-      const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
+      const float* yr = y_perm + static_cast<size_t>(r) * d + c;
+      const float4 y0 = __ldg(reinterpret_cast<const float4*>(yr));
+      const float4 y1 = __ldg(reinterpret_cast<const float4*>(yr + 4));
+      const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(g, bf16_bits_to_float(yw[i] & 0xFFFF), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(g, bf16_bits_to_float(yw[i] >> 16), acc[2 * i + 1]);
-      }
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, yv[i], acc[i]);
     }
     uint4 o;
     o.x = float_to_bf16_bits(acc[0]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[1])) << 16);
@@ -104,7 +104,7 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
 
 }  // namespace moe
 
-extern "C" int moe_combine(const uint16_t* u, const uint16_t* y_perm, const uint16_t* y_shared,
+extern "C" int moe_combine(const uint16_t* u, const float* y_perm, const float* y_shared,
                            const int32_t* inv, const float* gates, int T, int K_r, int d,
                            uint16_t* out, void* stream) {
   using namespace moe;

@@ -30,7 +30,8 @@
 //            Epilogue: SwiGLU a = silu(G) * U, 1x128 requantisation to E4M3
 //            (the tile is exactly one 128-channel scale tile), written to H.
 //   phase 2: per tile (group g, 128 rows, 256 output channels):
-//            A = H, B = W_down rows, epilogue converts to bf16.
+//            A = H, B = W_down rows; the FP32 accumulators are stored as they
+//            are (the combine adds them to the residual and rounds once).
 // Tiles are numbered group-major (shared expert last), then row tile, then
 // column tile, and dealt round-robin to CTAs, so the CTAs running at the same
 // time share weight tiles and activation rows through L2.
@@ -66,8 +67,8 @@ struct Args {
   const float* s_down;
   uint8_t* H;
   float* Hs;
-  uint16_t* y_perm;
-  uint16_t* y_shared;
+  float* y_perm;
+  float* y_shared;
 };
 
 struct Smem {
@@ -380,18 +381,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         if (valid) {
-          uint16_t* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
-                                     : a.y_perm + static_cast<size_t>(tl.row0 + rr) * a.d;
-          uint4* dst = reinterpret_cast<uint4*>(yrow + tl.n * BN + half * 128);
+          float* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
+                                  : a.y_perm + static_cast<size_t>(tl.row0 + rr) * a.d;
+          float4* dst = reinterpret_cast<float4*>(yrow + tl.n * BN + half * 128);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              w[k] = float_to_bf16_bits(acc[i * 8 + 2 * k]) |
-                     (static_cast<uint32_t>(float_to_bf16_bits(acc[i * 8 + 2 * k + 1])) << 16);
-            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
+          for (int i = 0; i < 32; ++i)
+            dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         }
       }
     }
@@ -421,7 +416,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
                                     int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
                                     const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
                                     const float* s_gate, const float* s_up, const float* s_down, int d,
-                                    int I, uint16_t* y_perm, uint16_t* y_shared, void* workspace,
+                                    int I, float* y_perm, float* y_shared, void* workspace,
                                     size_t ws_bytes, void* stream) {
   using namespace moe;
   using namespace moe::gg;

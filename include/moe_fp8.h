@@ -167,7 +167,7 @@ MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
  * shared expert (slot N_r, all T rows of xq):
  *   G = X W_gate^T, U = X W_up^T      (FP8 x FP8 -> FP32)
  *   A = silu(G) * U,  H = quant_1x128(A)
- *   Y = H W_down^T -> bf16
+ *   Y = H W_down^T, stored in FP32
  * Each product is sum over 128-wide K blocks kb of
  *   s_X[m,kb] * s_W[n/128,kb] * (X_kb . W_kb),
  * the block partial coming from the tensor cores and the scaling and the sum
@@ -177,7 +177,8 @@ MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
  *   xq, xs            [T][d], [T][d/128]: the shared expert's input
  *   w_gate, w_up      [N_r+1][I][d] E4M3;  s_gate, s_up  [N_r+1][I/128][d/128]
  *   w_down            [N_r+1][d][I] E4M3;  s_down        [N_r+1][d/128][I/128]
- *   y_perm            [P][d] bf16 (out)    y_shared [T][d] bf16 (out)
+ *   y_perm            [P][d] FP32 (out)    y_shared [T][d] FP32 (out)
+ *                     (FP32 so that h' is rounded to bf16 once, in moe_combine)
  *   workspace         moe_grouped_gemm_fp8_workspace(T, K_r, d, I) bytes
  * Limits: d a multiple of 256, I a multiple of 128, N_r <= 1024.
  */
@@ -187,19 +188,19 @@ MOE_API int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm,
                          const uint8_t* w_gate, const uint8_t* w_up,
                          const uint8_t* w_down, const float* s_gate,
                          const float* s_up, const float* s_down, int d, int I,
-                         uint16_t* y_perm, uint16_t* y_shared,
+                         float* y_perm, float* y_shared,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
  * ("DeepSeek-V3 Teknik Raporu", Yöntem 2, the h'_t equation). The sum is FP32
  * in the fixed order u, shared, k = 0..K_r-1.
- *   u, y_shared [T][d] bf16;  y_perm [T*K_r][d] bf16;  inv, gates [T][K_r]
+ *   u [T][d] bf16;  y_shared [T][d] FP32;  y_perm [T*K_r][d] FP32;  inv, gates [T][K_r]
  *   out [T][d] bf16 (may alias u)
  * d must be a multiple of 8.
  */
-MOE_API int moe_combine(const uint16_t* u, const uint16_t* y_perm,
-                const uint16_t* y_shared, const int32_t* inv,
+MOE_API int moe_combine(const uint16_t* u, const float* y_perm,
+                const float* y_shared, const int32_t* inv,
                 const float* gates, int T, int K_r, int d, uint16_t* out,
                 void* stream);
 

@@ -190,7 +190,7 @@ def expert_ffn(xq, xs, w: dict):
     a = silu(G) * U
     hq, hs = quant_1x128(round_fp32(a))
     Y = scaled_gemm(hq, hs, w["down_q"], w["down_s"])
-    return round_bf16(Y), dequant_1x128(hq, hs)
+    return Y, dequant_1x128(hq, hs)
 
 
 # --------------------------------------------------------------------------

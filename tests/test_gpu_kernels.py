@@ -177,8 +177,8 @@ def test_combine(lib, T, K, d):
     from fine_grained_fp8_sigmoid_b200 import binding as B
     g = torch.Generator().manual_seed(T + d)
     u = torch.randn(T, d, generator=g).to(torch.bfloat16)
-    ysh = (torch.randn(T, d, generator=g) * 0.1).to(torch.bfloat16)
-    yp = (torch.randn(T * K, d, generator=g) * 0.1).to(torch.bfloat16)
+    ysh = torch.randn(T, d, generator=g) * 3.0
+    yp = torch.randn(T * K, d, generator=g) * 3.0
     inv = torch.randperm(T * K, generator=g).reshape(T, K).to(torch.int32)
     gt = torch.rand(T, K, generator=g)
     gt = gt / gt.sum(dim=1, keepdim=True)
@@ -254,8 +254,8 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
     wg, wu, wd = stack("gate_q", torch.uint8), stack("up_q", torch.uint8), stack("down_q", torch.uint8)
     sg, su, sd = stack("gate_s", torch.float32), stack("up_s", torch.float32), stack("down_s", torch.float32)
     off = torch.from_numpy(offsets).cuda()
-    y_perm = torch.empty(Ppad, d, dtype=torch.bfloat16, **dev)
-    y_sh = torch.empty(T, d, dtype=torch.bfloat16, **dev)
+    y_perm = torch.empty(Ppad, d, dtype=torch.float32, **dev)
+    y_sh = torch.empty(T, d, dtype=torch.float32, **dev)
     ws = torch.empty(B.moe_grouped_gemm_fp8_workspace(T, K_r, d, I), dtype=torch.uint8, **dev)
     B.moe_grouped_gemm_fp8(xq_pd, xs_pd, off, cu(xq, torch.uint8), cu(xs, torch.float32),
                            wg, wu, wd, sg, su, sd, y_perm, y_sh, ws)

@@ -252,7 +252,7 @@ def _const_expert(d, I, gate_code, up_code, down_code):
 def test_expert_ffn_closed_form():
     # x = 1 (code 0x38, scale 1), all weights 2^-7 (code 0x04):
     # G = U = d * 2^-7 = 1 for d = 128, a = silu(1), requant maps a to 448 * scale,
-    # y = I * 2^-7 * 448 * scale = 448 * scale for I = 128.
+    # y = I * 2^-7 * 448 * scale = 448 * scale for I = 128 (exact: y is not rounded).
     d = I = 128
     xq = np.full((3, d), 0x38, np.uint8)
     xs = np.ones((3, 1))
@@ -260,7 +260,7 @@ def test_expert_ffn_closed_form():
     a = float(np.float32(1.0 / (1.0 + math.exp(-1.0))))
     scale = float(np.float32(a / 448.0))
     assert np.all(h == 448.0 * scale)
-    assert np.all(y == round_bf16(np.array([448.0 * scale]))[0])
+    assert np.all(y == 448.0 * scale)
 
 
 def test_expert_ffn_zero_gate_gives_zero():
@@ -352,7 +352,8 @@ def test_token_sample_matches_full_forward():
     tok = np.array([0, 5, 17, 63])
     part = moe.moe_forward(u, e, b, cfg.K_r, prov, tokens=tok)
     assert np.array_equal(part["out"], full["out"][tok])
-    assert np.array_equal(part["y_shared"], full["y_shared"][tok])
+    # up to float64 rounding order (the matmul blocks differently per batch size)
+    assert np.allclose(part["y_shared"], full["y_shared"][tok], rtol=1e-12, atol=1e-12)
     assert np.array_equal(part["bias_new"], full["bias_new"])
     # routed outputs sit where the permutation says
     assert full["counts"].sum() == cfg.T * cfg.K_r
