@@ -52,8 +52,14 @@ def layer_flops(cfg, rows_routed=None):
     return 6.0 * cfg.d * cfg.I * (P + cfg.T)
 
 
+def weight_bytes(cfg):
+    """E4M3 codes plus FP32 block scales of all N_r + 1 experts."""
+    per = 3 * cfg.d * cfg.I + 3 * (cfg.d // 128) * (cfg.I // 128) * 4
+    return (cfg.N_r + 1) * per
+
+
 def workload_desc(cfg):
-    return (f"DeepSeek-V3 MoE layer, prefill: T={cfg.T}, d={cfg.d}, {cfg.N_r} routed experts "
+    return (f"DeepSeek-V3 MoE layer, {cfg.name}: T={cfg.T}, d={cfg.d}, {cfg.N_r} routed experts "
             f"top-{cfg.K_r} + 1 shared, SwiGLU I={cfg.I}, E4M3 1x128/128x128 scales")
 
 
@@ -177,7 +183,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = workloads.CONFIGS[CONFIG_NAME]
+    cfg = workloads.CONFIGS[args.workload]
     peaks = _peaks()
 
     layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, device=dev)
@@ -285,7 +291,8 @@ def run_ours(args, rank, world, local_rank):
             "config": {"workload": workload_desc(cfg), "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r,
                        "K_r": cfg.K_r, "I": cfg.I, "N_s": 1, "seed": cfg.seed,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2: 11.3 GB of expert weights stream every step"},
+                       "l2": f"inputs larger than L2: {weight_bytes(cfg) / 1e9:.2f} GB of expert "
+                             "weights stream every step"},
             "tflops": layer_tf,
             "pct_fp8_peak": layer_tf / fp8_peak,
             "roofline": {"bound": "tensor", "kernel": "moe_grouped_gemm_fp8 (2 launches)",
@@ -344,6 +351,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=CONFIG_NAME,
+                    help="prefill (the benchmark) or a smaller layer for profiling: mid, decode, tiny")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
