@@ -106,6 +106,28 @@ def moe_permute(topk_idx, N_r, counts, offsets, sorted_token, inv, workspace,
         _stream(stream)))
 
 
+def moe_permute_noalloc(topk_idx, N_r, counts, offsets, sorted_token, inv,
+                        xq=None, xs=None, xq_perm=None, xs_perm=None, stream=None):
+    """moe_permute without a workspace: the library's static scratch array is
+    used instead (for callers that cannot allocate device memory)."""
+    T, K_r = topk_idx.shape
+    _want(topk_idx, torch.int32, (T, K_r), "topk_idx")
+    _want(counts, torch.int32, (N_r,), "counts")
+    _want(offsets, torch.int32, (N_r + 1,), "offsets")
+    _want(sorted_token, torch.int32, (T * K_r,), "sorted_token")
+    _want(inv, torch.int32, (T, K_r), "inv")
+    d = 0
+    if xq is not None:
+        d = xq.shape[1]
+        _want(xq, torch.uint8, (T, d), "xq")
+        _want(xs, torch.float32, (T, d // 128), "xs")
+        _want(xq_perm, torch.uint8, (T * K_r, d), "xq_perm")
+        _want(xs_perm, torch.float32, (T * K_r, d // 128), "xs_perm")
+    check("moe_permute_noalloc", _lib.load().moe_permute_noalloc(
+        _ptr(topk_idx), T, K_r, N_r, _ptr(xq), _ptr(xs), d, _ptr(counts), _ptr(offsets),
+        _ptr(sorted_token), _ptr(inv), _ptr(xq_perm), _ptr(xs_perm), _stream(stream)))
+
+
 def moe_grouped_gemm_fp8_workspace(T, K_r, d, I):
     return int(_lib.load().moe_grouped_gemm_fp8_workspace(T, K_r, d, I))
 

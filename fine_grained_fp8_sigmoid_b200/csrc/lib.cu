@@ -3,5 +3,6 @@
 #include "quant.cu"
 #include "route.cu"
 #include "permute.cu"
+#include "permute_noalloc.cu"
 #include "gemm.cu"
 #include "combine.cu"

@@ -155,6 +155,29 @@ MOE_API int moe_permute(const int32_t* topk_idx, int T, int K_r, int N_r,
                 void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_permute_noalloc: moe_permute for callers that cannot allocate device
+ * memory (no workspace argument). The pages have no counterpart: this is a
+ * deployment variant, not a step of the method. Same arguments, outputs and
+ * limits as moe_permute, minus workspace/ws_bytes. Its scratch is a static
+ * 1 MiB device array inside the library, held by every GPU that loads the
+ * library until the process exits.
+ *   - Sizes whose scratch (moe_permute_workspace(T, N_r)) exceeds 1 MiB are
+ *     rejected with MOE_ERR_UNSUPPORTED (moe_last_error_detail says why).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (different
+ *     streams, or different host threads, on the same device) race and must
+ *     be serialised by the caller. Nothing needs clearing between calls.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int K_r, int N_r,
+                        const uint8_t* xq, const float* xs, int d,
+                        int32_t* counts, int32_t* offsets, int32_t* sorted_token,
+                        int32_t* inv, uint8_t* xq_perm, float* xs_perm,
+                        void* stream);
+
+/*
  * moe_grouped_gemm_fp8_workspace: bytes of scratch for the intermediate
  * H = requant(SwiGLU(...)) of P = T*K_r routed rows plus T shared rows:
  * (P + T) * I bytes of E4M3 and (P + T) * I/128 FP32 scales.
