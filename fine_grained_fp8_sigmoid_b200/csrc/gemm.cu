@@ -16,7 +16,7 @@
 //
 // Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0     TMA producer: A tile 128 x 128 and B tile 256 x 128 per K block
-//              (128-byte swizzle), 4-stage ring.
+//              (128-byte swizzle), 4-stage ring (3 in phase 2).
 //   warp 1     MMA issuer (one thread) and TMEM owner (512 columns = 2 x 256).
 //   warps 2-3  idle (they complete the first warpgroup).
 //   warps 4-11 epilogue: warp w reads TMEM lanes 32*(w%4).. (rows), and
@@ -30,11 +30,18 @@
 //            Epilogue: SwiGLU a = silu(G) * U, 1x128 requantisation to E4M3
 //            (the tile is exactly one 128-channel scale tile), written to H.
 //   phase 2: per tile (group g, 128 rows, 256 output channels):
-//            A = H, B = W_down rows; the FP32 accumulators are stored as they
-//            are (the combine adds them to the residual and rounds once).
+//            A = H, B = W_down rows; the FP32 accumulators leave through
+//            shared memory and TMA stores (the combine adds them to the
+//            residual and rounds once).
 // Tiles are numbered group-major (shared expert last), then row tile, then
 // column tile, and dealt round-robin to CTAs, so the CTAs running at the same
 // time share weight tiles and activation rows through L2.
+//
+// The per-tile epilogue tail sits between two tiles' K loops, and the MMAs can
+// only run two K blocks ahead of it, so it is kept short: SwiGLU and the
+// requantisation use the fast exponential/division (branch-free, a few
+// instructions each, so the unrolled tail stays small), and the phase-2
+// output is handed to TMA instead of 32 scattered stores per thread.
 #include "host.cuh"
 
 namespace moe {
@@ -43,12 +50,12 @@ namespace gg {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 384;
 constexpr int EPI_THREADS = 256;
+constexpr int EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 4;     // first epilogue warp
 // launch at 168 registers (65536 / 384, rounded down to 8); then
 // 128 * 56 + 256 * 224 = 384 * 168, and 56 + 2 * 224 <= 512 per sub-partition
@@ -56,6 +63,16 @@ constexpr uint32_t REGS_CTRL = 56;
 constexpr uint32_t REGS_EPI = 224;
 constexpr int MAX_GROUPS = 1025;
 constexpr uint32_t TMEM_COLS = 512;
+// phase-2 output staging: per epilogue warp two 32 x 32 FP32 boxes
+constexpr int Y_BOX = 32;
+constexpr int Y_BOX_BYTES = Y_BOX * Y_BOX * 4;
+constexpr int Y_STAGING_BYTES = EPI_WARPS * 2 * Y_BOX_BYTES;
+
+template <int PHASE>
+struct Cfg {
+  static constexpr int STAGES = PHASE == 1 ? 4 : 3;
+  static constexpr int STAGING = PHASE == 1 ? 0 : Y_STAGING_BYTES;
+};
 
 struct Args {
   const int32_t* offsets;
@@ -71,6 +88,7 @@ struct Args {
   float* y_shared;
 };
 
+template <int STAGES>
 struct Smem {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -86,7 +104,10 @@ struct Smem {
   float amax_x[2][2][BM];  // [tile parity][column half][row]
 };
 
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + sizeof(Smem);
+template <int PHASE>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<PHASE>::STAGES * STAGE_BYTES + Cfg<PHASE>::STAGING + sizeof(Smem<Cfg<PHASE>::STAGES>);
+}
 
 __device__ __forceinline__ int find_group(const int* start, int G, int t) {
   int lo = 0, hi = G - 1;
@@ -102,8 +123,8 @@ struct Tile {
   bool shared;
 };
 
-template <int PHASE>
-__device__ __forceinline__ Tile decode_tile(const Smem& sm, const Args& a, int t, int n_tiles) {
+template <int PHASE, typename S>
+__device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, int n_tiles) {
   Tile tl;
   const int G = a.N_r + 1;
   tl.g = find_group(sm.tile_start, G, t);
@@ -121,16 +142,35 @@ __device__ __forceinline__ Tile decode_tile(const Smem& sm, const Args& a, int t
   return tl;
 }
 
-__device__ __forceinline__ float silu(float x) { return __fdiv_rn(x, 1.0f + expf(-x)); }
+// silu(x) = x / (1 + e^-x) with the fast exponential and division: branch-free
+// (x -> -inf gives e^-x = inf and x / inf = -0, the limit).
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// 2-D tiled store of one box from shared memory (bulk async group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(m),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N bulk groups of this thread still read shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int PHASE>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                        const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_ys,
                         const Args a) {
+  constexpr int STAGES = Cfg<PHASE>::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Smem& sm = *reinterpret_cast<Smem*>(tiles + STAGES * STAGE_BYTES);
+  uint8_t* staging = tiles + STAGES * STAGE_BYTES;   // 1024-aligned (phase 2 only)
+  Smem<STAGES>& sm = *reinterpret_cast<Smem<STAGES>*>(staging + Cfg<PHASE>::STAGING);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
@@ -146,10 +186,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.tfull[b], 1);
-      mbar_init(&sm.tempty[b], EPI_THREADS / 32);
+      mbar_init(&sm.tempty[b], EPI_WARPS);
     }
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.xbar, EPI_THREADS);
+    mbar_init(&sm.xbar, EPI_WARPS);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -195,11 +235,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = sm.tmem_base;
   const int total = sm.total_tiles;
   volatile int* abort = &sm.abort;
-  if (warp < EPI_WARP0) regs_decrease<REGS_CTRL>();
 
-  if (warp == 0) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp < EPI_WARP0) {
+    regs_decrease<REGS_CTRL>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------ TMA producer
       int armed[STAGES];
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
       int stage = 0;
@@ -234,10 +274,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int s = 0; s < STAGES; ++s)
           if (armed[s] >= 0) mbar_wait(&sm.full[s], armed[s], &never, 100000000ull);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------ MMA issuer
       const uint32_t idesc = make_idesc(0, 0, BM, BN);
       int stage = 0;
       uint32_t phase = 0;
@@ -269,11 +307,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       volatile int never = 0;
       mbar_wait(&sm.drain, 0, &never, 100000000ull);
     }
-  } else if (warp >= EPI_WARP0) {
+  } else {
     // ------------------------------------------------ epilogue
     regs_increase<REGS_EPI>();
+    const int ew = warp - EPI_WARP0;
     const int q = warp & 3;
-    const int half = (warp - EPI_WARP0) >> 2;
+    const int half = ew >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     int buf = 0;
@@ -351,18 +390,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         float amax = 0.0f;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          const float x = silu(acc[j]) * acc[64 + j];
+          const float x = silu_fast(acc[j]) * acc[64 + j];
           acc[j] = x;
           amax = fmaxf(amax, fabsf(x));
         }
         // exchange through shared memory, double-buffered by tile parity; the
         // mbarrier wait is bounded like every other wait here
         sm.amax_x[xpar][half][r] = amax;
-        mbar_arrive(&sm.xbar);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xbar);
         if (!warp_wait(&sm.xbar, xpar, abort)) break;
         amax = fmaxf(amax, sm.amax_x[xpar][half ^ 1][r]);
         xpar ^= 1;
+        // the scale follows the stored rule; the codes use one reciprocal of
+        // it (an E4M3 code can differ from dividing only when x/scale is
+        // within an FP32 ulp of a rounding midpoint)
         const float s = tile_scale(amax);
+        const float inv = __fdiv_rn(1.0f, s);
         if (valid) {
           const size_t hrow = static_cast<size_t>(tl.shared ? a.P + rr : tl.row0 + rr);
           uint4* dst = reinterpret_cast<uint4*>(a.H + hrow * a.I + tl.n * 128 + half * 64);
@@ -372,24 +416,56 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int j = i * 16 + k * 4;
-              w[k] = e4m3x2(__fdiv_rn(acc[j], s), __fdiv_rn(acc[j + 1], s)) |
-                     (e4m3x2(__fdiv_rn(acc[j + 2], s), __fdiv_rn(acc[j + 3], s)) << 16);
+              w[k] = e4m3x2(acc[j] * inv, acc[j + 1] * inv) | (e4m3x2(acc[j + 2] * inv, acc[j + 3] * inv) << 16);
             }
             dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
           if (half == 0) a.Hs[hrow * KBi + tl.n] = s;
         }
       } else {
-        if (valid) {
+        // This warp's 32 rows x 128 columns. Rows wholly inside the group go
+        // out as four 32 x 32 FP32 boxes: each lane writes its row into a
+        // 128-byte-swizzled shared-memory box (16-byte chunk c of row r at
+        // chunk c ^ (r % 8): bank-conflict free), and lane 0 hands the box to
+        // a TMA store. Two boxes per warp alternate; a box is rewritten only
+        // after the store issued two boxes earlier has read it.
+        const int row_first = tl.m * BM + q * 32;             // within the group
+        const int nvalid = min(Y_BOX, tl.rows - row_first);
+        const int col0 = tl.n * BN + half * 128;
+        if (nvalid == Y_BOX) {
+          const CUtensorMap* ym = tl.shared ? &tm_ys : &tm_y;
+          const int ytop = tl.shared ? row_first : tl.row0 + row_first;
+          uint8_t* wstage = staging + ew * 2 * Y_BOX_BYTES;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint8_t* box = wstage + (c & 1) * Y_BOX_BYTES;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *reinterpret_cast<float4*>(box + lane * 128 + ((i ^ (lane & 7)) * 16)) =
+                  make_float4(acc[c * 32 + 4 * i], acc[c * 32 + 4 * i + 1], acc[c * 32 + 4 * i + 2],
+                              acc[c * 32 + 4 * i + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(ym, box, col0 + c * 32, ytop);
+              bulk_commit();
+            }
+          }
+        } else if (valid) {
           float* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
                                   : a.y_perm + static_cast<size_t>(tl.row0 + rr) * a.d;
-          float4* dst = reinterpret_cast<float4*>(yrow + tl.n * BN + half * 128);
+          float4* dst = reinterpret_cast<float4*>(yrow + col0);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         }
       }
+      // END_OF_EPILOGUE_TILE
     }
+    if (PHASE == 2 && lane == 0) bulk_wait_all();
+    // END_OF_EPILOGUE
   }
 
   tc_fence_before();
@@ -401,6 +477,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// 2-D row-major FP32 tensor stored in 32 x 32 boxes with the 128-byte swizzle.
+inline int make_tmap_y(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
+  return make_tmap_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols, Y_BOX, Y_BOX);
+}
 
 }  // namespace gg
 }  // namespace moe
@@ -438,7 +519,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   uint8_t* H = static_cast<uint8_t*>(workspace);
   float* Hs = reinterpret_cast<float*>(H + align256(static_cast<size_t>(rowsH) * I));
 
-  CUtensorMap tmA, tmX, tmWg, tmWu, tmH, tmWd;
+  CUtensorMap tmA, tmX, tmWg, tmWu, tmH, tmWd, tmY, tmYs;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   if (int st = make_tmap_2d(&tmA, xq_perm, U8, 1, P, d, BM, BK)) return st;
   if (int st = make_tmap_2d(&tmX, xq, U8, 1, T, d, BM, BK)) return st;
@@ -446,6 +527,8 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = make_tmap_2d(&tmWu, w_up, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
   if (int st = make_tmap_2d(&tmH, H, U8, 1, rowsH, I, BM, BK)) return st;
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
+  if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
+  if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
 
   Args args;
   args.offsets = offsets;
@@ -472,14 +555,15 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
 
   auto k1 = grouped_gemm_kernel<1>;
   auto k2 = grouped_gemm_kernel<2>;
-  if (int st = cuda_status(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(SMEM_BYTES)), "smem attribute (gate/up)"))
+  constexpr size_t sm1 = smem_bytes<1>(), sm2 = smem_bytes<2>();
+  if (int st = cuda_status(cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm1)),
+                           "smem attribute (gate/up)"))
     return st;
-  if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(SMEM_BYTES)), "smem attribute (down)"))
+  if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
+                           "smem attribute (down)"))
     return st;
-  k1<<<g1, THREADS, SMEM_BYTES, s>>>(tmA, tmX, tmWg, tmWu, args);
+  k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
-  k2<<<g2, THREADS, SMEM_BYTES, s>>>(tmH, tmH, tmWd, tmWd, args);
+  k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, args);
   return launch_status("grouped GEMM launch (down)");
 }
