@@ -45,6 +45,22 @@ def _peaks():
         return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's value (every rank calls this at the same point)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens of all replicas per second, timed by the slowest rank."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def layer_flops(cfg, rows_routed=None):
     """Algorithmic FLOPs of the expert GEMMs: 6*d*I per (token, expert) pair
     (gate, up, down), routed pairs plus the shared expert on every token."""
@@ -229,16 +245,12 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ms_total = start.elapsed_time(stop)
+    ms_total = max_over_ranks(start.elapsed_time(stop), dev)
     gemm_ms = [a.elapsed_time(z) for a, z in ev]
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
     if B.moe_get_error() != 0:
         raise RuntimeError("device error word set during the timed region")
     ms_step = ms_total / K
-    tokens_per_s = world * cfg.T / (ms_step / 1e3)
+    tokens_per_s = whole_job_tokens_per_s(cfg.T, world, ms_step)
 
     flops = layer_flops(cfg)
     gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
@@ -261,12 +273,8 @@ def run_ours(args, rank, world, local_rank):
         layer.forward_host(u_host, e, b, out_host, u_dev)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / Ke
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_tps = world * cfg.T / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, dev)
+    e2e_tps = whole_job_tokens_per_s(cfg.T, world, e2e_ms)
 
     result = None
     if rank == 0:
@@ -322,18 +330,23 @@ def run_reference(args, rank, world):
     import numpy as np
     tokens = np.arange(n_tokens)
     u, e, b, quant = _oracle_sample_setup(cfg, tokens, device=dev)
-    for _ in range(args.warmup):
-        O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
+    for _ in range(max(1, args.warmup)):
         O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
-    dt = (time.perf_counter() - t0) / args.steps
+    one = (time.perf_counter() - t0) / max(1, args.warmup)
+    # the oracle is slow: run the requested steps, but no more than ~60 s of them
+    steps = max(1, min(args.steps, int(60.0 / max(one, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.moe_forward(u, e, b, cfg.K_r, quant.__getitem__)
+    dt = (time.perf_counter() - t0) / steps
     tps = n_tokens / dt
     desc = (f"oracle forward on token 0 of the {cfg.name} batch per step ({len(quant)} expert "
             f"FFNs incl. shared), weights pre-quantised by the oracle (inputs drawn on the CPU)")
     return {
         "impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "n_gpus": world, "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r,
