@@ -45,6 +45,24 @@ def _peaks():
         return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def gemm_traffic(cfg):
+    """DRAM bytes per moe_grouped_gemm_fp8 call from the committed ncu summary,
+    if it was taken on this workload with the current GEMM source; else None."""
+    import hashlib
+    import re
+    src = os.path.join(ROOT, "fine_grained_fp8_sigmoid_b200", "csrc", "gemm.cu")
+    prof = os.path.join(ROOT, "profiles", f"grouped_gemm_{cfg.name}_traffic.md")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        txt = open(prof).read()
+        if re.search(r"gemm_cu_sha256:\s*" + sha, txt) is None:
+            return None
+        m = re.search(r"dram_bytes_per_call:\s*([0-9.eE+]+)", txt)
+        return float(m.group(1)) if m else None
+    except OSError:
+        return None
+
+
 def max_over_ranks(value: float, device=None) -> float:
     """The slowest rank's value (every rank calls this at the same point)."""
     import torch
@@ -258,6 +276,20 @@ def run_ours(args, rank, world, local_rank):
     achieved_tf = flops / gemm_avg_s / 1e12
     layer_tf = flops / (ms_step / 1e3) / 1e12
 
+    balance = None
+    if cfg.name == "skew":
+        # the auxiliary-loss-free balancing run: 100 steps of route -> experts ->
+        # bias update from the initial bias, max/mean expert load of each step
+        b.copy_(b0)
+        ratios = torch.zeros(100, device=dev)
+        for i in range(100):
+            layer.forward(u, e, b, update_bias=True)
+            ratios[i].copy_(layer.max_over_mean[0])
+        r = ratios.cpu().tolist()
+        balance = {"steps": 100, "gamma": 0.001, "max_over_mean_first": r[0],
+                   "max_over_mean_last": r[-1], "max_over_mean_min": min(r),
+                   "max_over_mean_every_10": r[::10]}
+
     # end to end through the public API: pinned host u in, h' out, every step
     u_host = u.cpu().pin_memory()
     out_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
@@ -305,13 +337,14 @@ def run_ours(args, rank, world, local_rank):
             "pct_fp8_peak": layer_tf / fp8_peak,
             "roofline": {"bound": "tensor", "kernel": "moe_grouped_gemm_fp8 (2 launches)",
                          "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": achieved_tf / fp8_peak, "traffic": None,
+                         "frac": achieved_tf / fp8_peak, "traffic": gemm_traffic(cfg),
                          "peak_source": f"{peaks['source']} bf16 {peaks['bf16']} TF/s x2 (burst)",
                          "gemm_ms": float(np.mean(gemm_ms))},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tps, "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
             "gpu_launches": 10 * K,
+            "balance": balance,
             "clocks": clk.summary(),
         }
     return result
