@@ -5,30 +5,44 @@
 
 namespace moe {
 
-// One warp per 1x128 tile: each lane holds 4 consecutive bf16 (8 bytes), so a
-// warp reads 256 contiguous bytes and writes 128 bytes of codes.
+// Half a warp per 1x128 tile: each lane holds 8 consecutive bf16 (16 bytes),
+// so a warp reads 512 contiguous bytes (two tiles) per step and writes 256
+// bytes of codes; the max-abs is reduced over the 16 lanes of a tile.
 __global__ void __launch_bounds__(256) quant_1x128_kernel(const uint16_t* __restrict__ x,
                                                           long long n_tiles, int tiles_per_row,
                                                           uint8_t* __restrict__ q,
                                                           float* __restrict__ scale) {
   const int lane = lane_id();
+  const int sub = lane & 15;                 // lane within the tile
+  const long long n_pairs = (n_tiles + 1) / 2;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
-  for (long long tile = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); tile < n_tiles;
-       tile += warps) {
-    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(x + tile * 128) + lane);
-    float v[4];
-    v[0] = bf16_bits_to_float(raw.x & 0xFFFF);
-    v[1] = bf16_bits_to_float(raw.x >> 16);
-    v[2] = bf16_bits_to_float(raw.y & 0xFFFF);
-    v[3] = bf16_bits_to_float(raw.y >> 16);
-    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  for (long long pr = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); pr < n_pairs; pr += warps) {
+    const long long tile = pr * 2 + (lane >> 4);
+    const bool live = tile < n_tiles;         // the last pair may hold one tile
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (live) raw = __ldg(reinterpret_cast<const uint4*>(x + tile * 128) + sub);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_bits_to_float(w[i] & 0xFFFF);
+      v[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float s = tile_scale(amax);
-    const uint32_t lo = e4m3x2(__fdiv_rn(v[0], s), __fdiv_rn(v[1], s));
-    const uint32_t hi = e4m3x2(__fdiv_rn(v[2], s), __fdiv_rn(v[3], s));
-    reinterpret_cast<uint32_t*>(q + tile * 128)[lane] = lo | (hi << 16);
-    if (lane == 0) scale[tile] = s;  // tiles are numbered row-major: [row][col/128]
+    uint32_t c[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+      c[i] = e4m3x2(__fdiv_rn(v[4 * i], s), __fdiv_rn(v[4 * i + 1], s)) |
+             (e4m3x2(__fdiv_rn(v[4 * i + 2], s), __fdiv_rn(v[4 * i + 3], s)) << 16);
+    if (live) {
+      reinterpret_cast<uint2*>(q + tile * 128)[sub] = make_uint2(c[0], c[1]);
+      if (sub == 0) scale[tile] = s;          // tiles are numbered row-major: [row][col/128]
+    }
   }
   (void)tiles_per_row;
 }
@@ -84,11 +98,11 @@ extern "C" int moe_quant_1x128(const uint16_t* x, int rows, int cols, uint8_t* q
   MOE_CHECK_SUPPORTED(cols % 128 == 0);
   if (rows == 0 || cols == 0) return MOE_OK;
   MOE_CHECK_ARG(x && q && scale);
-  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(x) % 8 == 0 && reinterpret_cast<uintptr_t>(q) % 4 == 0);
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(x) % 16 == 0 && reinterpret_cast<uintptr_t>(q) % 8 == 0);
   DeviceInfo di;
   if (int st = device_info(&di)) return st;
   const long long n_tiles = static_cast<long long>(rows) * (cols / 128);
-  long long blocks = (n_tiles + 7) / 8;
+  long long blocks = (n_tiles + 15) / 16;   // 8 warps of two tiles each
   const long long cap = static_cast<long long>(di.sm_count) * 16;
   if (blocks > cap) blocks = cap;
   quant_1x128_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(

@@ -9,8 +9,12 @@
 // (BF16 x BF16 -> FP32) write a fresh TMEM partial, and the epilogue warps add
 // the partials in FP32 registers. Accumulating all of d = 7168 inside the
 // tensor core lets its truncating accumulation drift by ~1e-4 in the logit;
-// summing 64-wide partials in registers keeps the error near FP32 rounding,
-// the same promotion the FP8 GEMMs use.
+// each TMEM partial here covers RK = 4 K blocks (256 channels) and the
+// epilogue adds the partials in FP32 registers, which keeps the error near
+// FP32 rounding while reading the 128 x 256 partial back only every fourth
+// K block (the read-back competes with the MMAs for TMEM).
+// After the K loop the logits are parked in the (now idle) pipeline shared
+// memory, so sigmoid and the top-K insertion run as a compact rolled loop.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
 // epilogue (TMEM lane quadrant w%4, column half (w-4)/4), which finishes
 // with sigmoid, the biased top-K of each half, and a merge of the halves.
@@ -23,6 +27,7 @@ constexpr int BM = 128;          // tokens per CTA (TMEM lanes)
 constexpr int BK = 64;           // bf16 per K block = 128 bytes = one swizzle row
 constexpr int NP = 256;          // MMA N: all experts of a token in one tile
 constexpr int STAGES = 4;
+constexpr int RK = 4;            // K blocks per TMEM partial
 constexpr int THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
@@ -174,12 +179,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     } else if (warp == 1 && lane == 0) {
       const uint32_t idesc = make_idesc(1, 1, BM, NP);
-      int buf = 0;
-      uint32_t tphase = 0;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) break;
+        const int grp = kb / RK;                 // partial buffer group
+        const int buf = grp & 1;
+        const bool first = kb % RK == 0, last = kb % RK == RK - 1 || kb == KB - 1;
+        if (first && !mbar_wait(&sm.tempty[buf], ((grp >> 1) & 1) ^ 1, abort)) break;
         if (!mbar_wait(&sm.full[s], ph, abort)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(tiles + s * STAGE_BYTES);
@@ -187,11 +193,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)  // 16 bf16 = 32 bytes per MMA
-          umma_f16(tmem + buf * NP, ad + 2 * k, bd + 2 * k, idesc, k != 0);
+          umma_f16(tmem + buf * NP, ad + 2 * k, bd + 2 * k, idesc, (k != 0) || !first);
         umma_commit(&sm.empty[s]);
-        umma_commit(&sm.tfull[buf]);
-        buf ^= 1;
-        if (buf == 0) tphase ^= 1;
+        if (last) umma_commit(&sm.tfull[buf]);
       }
       // all MMAs of this thread complete before TMEM is released
       umma_commit(&sm.drain);
@@ -208,11 +212,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     float acc[128];
 #pragma unroll
     for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
-    int buf = 0;
-    uint32_t tphase = 0;
     bool ok = true;
-    for (int kb = 0; kb < KB; ++kb) {
-      if (!warp_wait(&sm.tfull[buf], tphase, abort)) { ok = false; break; }
+    const int NG = (KB + RK - 1) / RK;
+    for (int grp = 0; grp < NG; ++grp) {
+      const int buf = grp & 1;
+      if (!warp_wait(&sm.tfull[buf], (grp >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -224,32 +228,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tempty[buf]);
-      buf ^= 1;
-      if (buf == 0) tphase ^= 1;
     }
     if (ok) {
+      // Every TMA load was consumed by an MMA and every MMA has completed
+      // (the last partial has been read), so the stage buffers are free:
+      // park this thread's 128 logits there, column-major so that a warp's
+      // accesses fall in consecutive banks, and walk them in a rolled loop.
+      float* park = reinterpret_cast<float*>(tiles) + half * 128 * BM;
+#pragma unroll
+      for (int j = 0; j < 128; ++j) park[j * BM + r] = acc[j];
       float kk[KMAX], ss[KMAX];
       int ii[KMAX];
       topk_init(kk, ii, ss);
-#pragma unroll
-      for (int j = 0; j < 128; ++j) {
+      const int ncol = min(128, N_r - half * 128);
+      float* srow = (scores_out != nullptr && t < T) ? scores_out + static_cast<size_t>(t) * N_r + half * 128 : nullptr;
+#pragma unroll 1
+      for (int j = 0; j < ncol; ++j) {
         const int col = half * 128 + j;
-        const float sg = sigmoidf(acc[j]);
-        acc[j] = sg;
-        if (col < N_r) topk_insert(kk, ii, ss, sg + sm.bias[col], col, sg);
-      }
-      if (scores_out != nullptr && t < T) {
-        float* dst = scores_out + static_cast<size_t>(t) * N_r + half * 128;
-        const int ncol = min(128, N_r - half * 128);
-        if ((N_r & 3) == 0 && ncol == 128) {
-#pragma unroll
-          for (int j = 0; j < 128; j += 4)
-            *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 128; ++j)
-            if (j < ncol) dst[j] = acc[j];
-        }
+        const float sg = sigmoidf(park[j * BM + r]);
+        topk_insert(kk, ii, ss, sg + sm.bias[col], col, sg);
+        if (srow != nullptr) srow[j] = sg;
       }
       // the upper half hands its list to the lower half, which merges: every
       // upper-half index exceeds every lower-half one, and the list arrives
