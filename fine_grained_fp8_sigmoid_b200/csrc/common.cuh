@@ -247,6 +247,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Issues a read of 8 consecutive FP32 columns of the thread's TMEM lane into
+// r[0..7] without waiting; the values are valid after tmem_wait_ld(r).
+__device__ __forceinline__ void tmem_ld8_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+
+// Waits for the thread's outstanding TMEM reads. Each register passes through
+// an empty asm placed after the wait, so no use of it can move above the wait.
+template <int N>
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[N]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Register budget changes for warp-specialised kernels (all threads of a
 // warpgroup execute them together). The values used with a launch of T
 // threads at R registers must satisfy: sum over warpgroups of 128 * regs <=

@@ -42,6 +42,8 @@
 // requantisation use the fast exponential/division (branch-free, a few
 // instructions each, so the unrolled tail stays small), and the phase-2
 // output is handed to TMA instead of 32 scattered stores per thread.
+#include <algorithm>
+
 #include "host.cuh"
 
 namespace moe {
@@ -77,6 +79,7 @@ struct Cfg {
 struct Args {
   const int32_t* offsets;
   int N_r, T, P, d, I;
+  int narrow_max;            // group remainders of 1..narrow_max rows go to the narrow kernel (0: none)
   const float* xs_perm;
   const float* xs;
   const float* s_gate;
@@ -109,6 +112,13 @@ constexpr size_t smem_bytes() {
   return 1024 + Cfg<PHASE>::STAGES * STAGE_BYTES + Cfg<PHASE>::STAGING + sizeof(Smem<Cfg<PHASE>::STAGES>);
 }
 
+// Rows at the end of a group of `rows` left to the narrow-tile kernel: the
+// remainder after whole 128-row tiles, when it is 1..narrow_max rows.
+__device__ __forceinline__ int narrow_part(int rows, int narrow_max) {
+  const int rem = rows % BM;
+  return rem <= narrow_max ? rem : 0;
+}
+
 __device__ __forceinline__ int find_group(const int* start, int G, int t) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {
@@ -139,6 +149,7 @@ __device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, i
     tl.row0 = sm.off[tl.g];
     tl.rows = sm.off[tl.g + 1] - tl.row0;
   }
+  tl.rows -= narrow_part(tl.rows, a.narrow_max);  // rows this kernel covers
   return tl;
 }
 
@@ -207,7 +218,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   for (int g = threadIdx.x; g < G; g += THREADS) {
     const int rows = g == a.N_r ? a.T : sm.off[g + 1] - sm.off[g];
-    sm.tile_start[g] = ((rows + BM - 1) / BM) * n_tiles;
+    const int wide = rows - narrow_part(rows, a.narrow_max);
+    sm.tile_start[g] = ((wide + BM - 1) / BM) * n_tiles;
   }
   __syncthreads();
   if (warp == 0) {  // exclusive prefix sum of tile counts, in place
@@ -486,6 +498,8 @@ inline int make_tmap_y(CUtensorMap* m, const float* base, uint64_t rows, uint64_
 }  // namespace gg
 }  // namespace moe
 
+#include "gemm_narrow.cu"
+
 extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
   (void)d;
   if (T <= 0 || K_r <= 0 || I <= 0) return 0;
@@ -529,6 +543,15 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
   if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
   if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
+  // narrow tiles: token operands in boxes of 64 rows, W_down in 128-row boxes
+  const bool narrow = d / BK <= gn::MAX_KB && I / BK <= gn::MAX_KB;
+  CUtensorMap tnX, tnXs, tnH, tnWd;
+  if (narrow) {
+    if (int st = make_tmap_2d(&tnX, xq_perm, U8, 1, P, d, gn::NMAX, BK)) return st;
+    if (int st = make_tmap_2d(&tnXs, xq, U8, 1, T, d, gn::NMAX, BK)) return st;
+    if (int st = make_tmap_2d(&tnH, H, U8, 1, rowsH, I, gn::NMAX, BK)) return st;
+    if (int st = make_tmap_2d(&tnWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, 128, BK)) return st;
+  }
 
   Args args;
   args.offsets = offsets;
@@ -546,6 +569,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   args.Hs = Hs;
   args.y_perm = y_perm;
   args.y_shared = y_shared;
+  args.narrow_max = narrow ? gn::NMAX : 0;
 
   // upper bound on row tiles: every non-empty routed group wastes < 1 tile
   const long long m_tiles = (P + BM - 1) / BM + (P < N_r ? P : N_r) + (T + BM - 1) / BM;
@@ -562,8 +586,30 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
                            "smem attribute (down)"))
     return st;
+  // narrow tiles: at most one per group and column tile
+  const int gn1 = std::min<long long>(di.sm_count, static_cast<long long>(N_r + 1) * (I / 128));
+  const int gn2 = std::min<long long>(di.sm_count, static_cast<long long>(N_r + 1) * (d / 256));
+  auto n1 = gn::narrow_gemm_kernel<1>;
+  auto n2 = gn::narrow_gemm_kernel<2>;
+  if (narrow) {
+    if (int st = cuda_status(cudaFuncSetAttribute(n1, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(gn::SMEM_BYTES)), "smem attribute (narrow gate/up)"))
+      return st;
+    if (int st = cuda_status(cudaFuncSetAttribute(n2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(gn::SMEM_BYTES)), "smem attribute (narrow down)"))
+      return st;
+  }
   k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
+  if (narrow) {
+    n1<<<gn1, gn::THREADS, gn::SMEM_BYTES, s>>>(tnX, tnXs, tmWg, tmWu, args);
+    if (int st = launch_status("narrow GEMM launch (gate/up)")) return st;
+  }
   k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, args);
-  return launch_status("grouped GEMM launch (down)");
+  if (int st = launch_status("grouped GEMM launch (down)")) return st;
+  if (narrow) {
+    n2<<<gn2, gn::THREADS, gn::SMEM_BYTES, s>>>(tnH, tnH, tnWd, tnWd, args);
+    if (int st = launch_status("narrow GEMM launch (down)")) return st;
+  }
+  return MOE_OK;
 }
