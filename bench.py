@@ -238,6 +238,7 @@ def run_ours(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+    gemm_launches = B.moe_grouped_gemm_fp8_launches(cfg.d, cfg.I)
     if B.moe_get_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
@@ -335,7 +336,7 @@ def run_ours(args, rank, world, local_rank):
                              "weights stream every step"},
             "tflops": layer_tf,
             "pct_fp8_peak": layer_tf / fp8_peak,
-            "roofline": {"bound": "tensor", "kernel": "moe_grouped_gemm_fp8 (2 launches)",
+            "roofline": {"bound": "tensor", "kernel": f"moe_grouped_gemm_fp8 ({gemm_launches} launches)",
                          "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
                          "frac": achieved_tf / fp8_peak, "traffic": gemm_traffic(cfg),
                          "peak_source": f"{peaks['source']} bf16 {peaks['bf16']} TF/s x2 (burst)",
@@ -343,7 +344,9 @@ def run_ours(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tps, "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
-            "gpu_launches": 10 * K,
+            # quant, router, permute (count, scan, scatter, gather), the GEMM's
+            # launches, combine, bias update
+            "gpu_launches": (8 + gemm_launches) * K,
             "balance": balance,
             "clocks": clk.summary(),
         }

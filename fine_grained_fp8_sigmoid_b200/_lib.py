@@ -31,6 +31,7 @@ SIGNATURES = {
     "moe_permute": (_i, [_p, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _z, _p]),
     "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p]),
     "moe_grouped_gemm_fp8_workspace": (_z, [_i, _i, _i, _i]),
+    "moe_grouped_gemm_fp8_launches": (_i, [_i, _i]),
     "moe_grouped_gemm_fp8": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p,
                                   _i, _i, _p, _p, _p, _z, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),

@@ -132,6 +132,10 @@ def moe_grouped_gemm_fp8_workspace(T, K_r, d, I):
     return int(_lib.load().moe_grouped_gemm_fp8_workspace(T, K_r, d, I))
 
 
+def moe_grouped_gemm_fp8_launches(d, I):
+    return int(_lib.load().moe_grouped_gemm_fp8_launches(d, I))
+
+
 def moe_grouped_gemm_fp8(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down,
                          s_gate, s_up, s_down, y_perm, y_shared, workspace, stream=None):
     T, d = xq.shape

@@ -507,6 +507,14 @@ extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
   return moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float);
 }
 
+// the narrow kernels need the tile's K-block factor table to fit shared memory
+static bool narrow_enabled(int d, int I) { return d / moe::gg::BK <= moe::gn::MAX_KB && I / moe::gg::BK <= moe::gn::MAX_KB; }
+
+extern "C" int moe_grouped_gemm_fp8_launches(int d, int I) {
+  if (d <= 0 || I <= 0) return -1;
+  return narrow_enabled(d, I) ? 4 : 2;
+}
+
 extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
                                     int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
                                     const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
@@ -544,7 +552,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
   if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
   // narrow tiles: token operands in boxes of 64 rows, W_down in 128-row boxes
-  const bool narrow = d / BK <= gn::MAX_KB && I / BK <= gn::MAX_KB;
+  const bool narrow = narrow_enabled(d, I);
   CUtensorMap tnX, tnXs, tnH, tnWd;
   if (narrow) {
     if (int st = make_tmap_2d(&tnX, xq_perm, U8, 1, P, d, gn::NMAX, BK)) return st;

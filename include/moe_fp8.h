@@ -185,6 +185,16 @@ MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int K_r, int N_r
 MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
 
 /*
+ * moe_grouped_gemm_fp8_launches: number of kernel launches one
+ * moe_grouped_gemm_fp8 call with these sizes makes on its stream (2, or 4
+ * when the narrow-tile kernels for groups of at most 64 rows are enabled:
+ * d/128 <= 56 and I/128 <= 56). A host-side query; no device work. The
+ * pages have no counterpart: it exists so that callers can account for
+ * launches. Returns -1 for non-positive sizes.
+ */
+MOE_API int moe_grouped_gemm_fp8_launches(int d, int I);
+
+/*
  * moe_grouped_gemm_fp8: every expert FFN of the layer on FP8 operands.
  * For routed expert i (rows offsets[i]..offsets[i+1] of xq_perm) and for the
  * shared expert (slot N_r, all T rows of xq):

@@ -53,6 +53,15 @@ def test_workspace_sizes(lib):
     assert ws == ((rows * 2048 + 255) // 256) * 256 + rows * 16 * 4
 
 
+def test_gemm_launch_count_query(lib):
+    # narrow-tile kernels only while a tile's factor table (56 K blocks) fits
+    assert lib.moe_grouped_gemm_fp8_launches(7168, 2048) == 4
+    assert lib.moe_grouped_gemm_fp8_launches(7168, 7168) == 4
+    assert lib.moe_grouped_gemm_fp8_launches(7424, 2048) == 2
+    assert lib.moe_grouped_gemm_fp8_launches(7168, 7296) == 2
+    assert lib.moe_grouped_gemm_fp8_launches(0, 2048) == -1
+
+
 def test_host_side_argument_checks(lib):
     N = None
     s = ctypes.c_void_p(0)
