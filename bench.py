@@ -45,15 +45,25 @@ def _peaks():
         return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
 
 
+def gemm_source_sha256(csrc):
+    """sha256 of the grouped GEMM's source (gemm.cu)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("gemm.cu",):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def gemm_traffic(cfg):
     """DRAM bytes per moe_grouped_gemm_fp8 call from the committed ncu summary,
     if it was taken on this workload with the current GEMM source; else None."""
     import hashlib
     import re
-    src = os.path.join(ROOT, "fine_grained_fp8_sigmoid_b200", "csrc", "gemm.cu")
+    csrc = os.path.join(ROOT, "fine_grained_fp8_sigmoid_b200", "csrc")
     prof = os.path.join(ROOT, "profiles", f"grouped_gemm_{cfg.name}_traffic.md")
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        sha = gemm_source_sha256(csrc)
         txt = open(prof).read()
         if re.search(r"gemm_cu_sha256:\s*" + sha, txt) is None:
             return None

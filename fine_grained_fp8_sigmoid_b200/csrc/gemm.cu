@@ -37,6 +37,15 @@
 // column tile, and dealt round-robin to CTAs, so the CTAs running at the same
 // time share weight tiles and activation rows through L2.
 //
+// Narrow tiles: a group of only 1..64 rows (decode batches: a few tokens per
+// expert) would pay a 128 x 256 partial read-back per K block for them. Its
+// tile swaps the MMA's roles instead: the two 128-row weight tiles of the
+// stage are M, the group's N = rows rounded up to 16 token rows are N (two
+// N <= 64 MMAs into columns 0 and 128 of the partial buffer), and the
+// epilogue owns one weight row per thread with a per-token scale table in
+// shared memory: half the TMEM read-back, and less power for the same
+// weight stream. Its TMA loads are the wide tile's.
+//
 // The per-tile epilogue tail sits between two tiles' K loops, and the MMAs can
 // only run two K blocks ahead of it, so it is kept short: SwiGLU and the
 // requantisation use the fast exponential/division (branch-free, a few
@@ -65,6 +74,12 @@ constexpr uint32_t REGS_CTRL = 56;
 constexpr uint32_t REGS_EPI = 224;
 constexpr int MAX_GROUPS = 1025;
 constexpr uint32_t TMEM_COLS = 512;
+// narrow tiles: at most 64 token rows; K blocks of the tile's token-scale
+// table (phase 1: d/128, phase 2: I/128; phase 2 has less room beside the
+// output staging)
+constexpr int NMAX = 64;
+constexpr int MAX_KB_N1 = 56;
+constexpr int MAX_KB_N2 = 24;
 // phase-2 output staging: per epilogue warp two 32 x 32 FP32 boxes
 constexpr int Y_BOX = 32;
 constexpr int Y_BOX_BYTES = Y_BOX * Y_BOX * 4;
@@ -74,12 +89,13 @@ template <int PHASE>
 struct Cfg {
   static constexpr int STAGES = PHASE == 1 ? 4 : 3;
   static constexpr int STAGING = PHASE == 1 ? 0 : Y_STAGING_BYTES;
+  static constexpr int TAB_KB = PHASE == 1 ? MAX_KB_N1 : MAX_KB_N2;
 };
 
 struct Args {
   const int32_t* offsets;
   int N_r, T, P, d, I;
-  int narrow_max;            // group remainders of 1..narrow_max rows go to the narrow kernel (0: none)
+  int narrow_max;            // groups of 1..narrow_max rows run as narrow tiles (0: none)
   const float* xs_perm;
   const float* xs;
   const float* s_gate;
@@ -91,32 +107,40 @@ struct Args {
   float* y_shared;
 };
 
-template <int STAGES>
+template <int STAGES, int TAB_KB>
 struct Smem {
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  uint64_t xbar;      // epilogue exchange of per-half max-abs (phase 1)
+  uint64_t xbar;      // epilogue exchange of max-abs partials (phase 1)
+  uint64_t sbar;      // narrow tile: token-scale table staged (8 warps)
+  uint64_t dbar;      // narrow tile: token-scale table no longer read (8 warps)
   uint32_t tmem_base;
   int abort;
   int total_tiles;
   int off[MAX_GROUPS + 1];
   int tile_start[MAX_GROUPS + 1];
-  float amax_x[2][2][BM];  // [tile parity][column half][row]
+  // wide tiles: [tile parity][column half][row]; narrow tiles use each
+  // parity's 256 floats as [lane quadrant][token]
+  float amax_x[2][2][BM];
+  alignas(16) float xs_tab[TAB_KB][NMAX];  // narrow tile: [kb][token] activation scales
 };
 
 template <int PHASE>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<PHASE>::STAGES * STAGE_BYTES + Cfg<PHASE>::STAGING + sizeof(Smem<Cfg<PHASE>::STAGES>);
+  return 1024 + Cfg<PHASE>::STAGES * STAGE_BYTES + Cfg<PHASE>::STAGING +
+         sizeof(Smem<Cfg<PHASE>::STAGES, Cfg<PHASE>::TAB_KB>);
 }
+static_assert(smem_bytes<1>() <= 227 * 1024 && smem_bytes<2>() <= 227 * 1024, "shared memory per CTA");
 
-// Rows at the end of a group of `rows` left to the narrow-tile kernel: the
-// remainder after whole 128-row tiles, when it is 1..narrow_max rows.
+// Rows of a group that form a narrow tile: the whole group when it has
+// 1..narrow_max rows. (Measured: a narrow tile for the remainder of a larger
+// group is no cheaper than the padded 128-row tile, since an MMA with N <= 64
+// costs nearly as much as one with N = 256.)
 __device__ __forceinline__ int narrow_part(int rows, int narrow_max) {
-  const int rem = rows % BM;
-  return rem <= narrow_max ? rem : 0;
+  return rows <= narrow_max ? rows : 0;
 }
 
 __device__ __forceinline__ int find_group(const int* start, int G, int t) {
@@ -130,7 +154,8 @@ __device__ __forceinline__ int find_group(const int* start, int G, int t) {
 
 struct Tile {
   int g, m, n, rows, row0;  // rows of the group; row0 = first row of the group in its A tensor
-  bool shared;
+  int mrows;                // narrow tile: its rows (1..narrow_max, the whole group)
+  bool shared, narrow;
 };
 
 template <int PHASE, typename S>
@@ -149,7 +174,8 @@ __device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, i
     tl.row0 = sm.off[tl.g];
     tl.rows = sm.off[tl.g + 1] - tl.row0;
   }
-  tl.rows -= narrow_part(tl.rows, a.narrow_max);  // rows this kernel covers
+  tl.mrows = narrow_part(tl.rows, a.narrow_max);  // a narrow group has one row tile
+  tl.narrow = tl.mrows > 0;
   return tl;
 }
 
@@ -171,6 +197,172 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+// acc[i] += fl32(t_i * w) * r[i] for four consecutive values (t: staged
+// activation scales, w: the weight block's scale; the factor is rounded to
+// FP32 before the FMA, as in the wide tiles)
+__device__ __forceinline__ void fma4(float* acc, const float4 t, float w, const uint32_t* r) {
+  acc[0] = fmaf(t.x * w, __uint_as_float(r[0]), acc[0]);
+  acc[1] = fmaf(t.y * w, __uint_as_float(r[1]), acc[1]);
+  acc[2] = fmaf(t.z * w, __uint_as_float(r[2]), acc[2]);
+  acc[3] = fmaf(t.w * w, __uint_as_float(r[3]), acc[3]);
+}
+
+struct NarrowCtx {
+  uint32_t tq;                  // TMEM address of the warp's lane quadrant, column 0
+  int q, half, lane, tid, KB;   // tid: 0..255 over the epilogue warps
+  volatile int* abort;
+};
+
+// Epilogue of a narrow tile: a group of 1..64 rows, computed with the
+// weights as the MMA's M side, so TMEM lane = weight row (channel) and TMEM
+// column = token. N = 2 * NC token columns (the rows rounded up to 16).
+//   phase 1: columns [0, N) hold W_gate x X^T and [128, 128 + N) W_up x X^T of
+//            the tile's 128 channels; the thread (channel c) owns tokens
+//            half*NC .. +NC of both, pairs them in SwiGLU and requantises each
+//            token's 128 channels (max-abs across lanes, then across the four
+//            lane-quadrant warps).
+//   phase 2: columns [half*128, half*128 + N) hold W_down rows n*256 +
+//            half*128 .. +128 x H^T; the thread owns all N tokens of one
+//            output channel.
+// The activation scales of the tile are staged once per tile as a [kb][token]
+// table, so each value costs one FP32 multiply and one FMA.
+template <int PHASE, int NC, typename S>
+__device__ __forceinline__ bool narrow_tile(S& sm, const Args& a, const Tile tl, const NarrowCtx x, int& buf,
+                                            uint32_t& tphase, uint32_t& xpar, int& nn) {
+  constexpr int NV = 2 * NC;
+  const int KBd = a.d / BK, KBi = a.I / BK;
+  const int r0 = tl.row0 + tl.m * BM;   // first row of the tile in the A tensor
+
+  // stage the table once the previous narrow tile's table is read by all warps
+  if (nn > 0 && !warp_wait(&sm.dbar, (nn - 1) & 1, x.abort)) return false;
+  {
+    const float* xsrc = PHASE == 1 ? (tl.shared ? a.xs : a.xs_perm) + static_cast<size_t>(r0) * KBd
+                                   : a.Hs + static_cast<size_t>(r0) * KBi;
+    for (int e = x.tid; e < x.KB * NMAX; e += EPI_THREADS) {
+      const int kb = e / NMAX, j = e % NMAX;
+      sm.xs_tab[kb][j] = j < tl.mrows ? __ldg(xsrc + static_cast<size_t>(j) * x.KB + kb) : 0.0f;
+    }
+  }
+  __syncwarp();
+  if (x.lane == 0) mbar_arrive(&sm.sbar);
+  if (!warp_wait(&sm.sbar, nn & 1, x.abort)) return false;
+  ++nn;
+
+  const int j0 = PHASE == 1 ? x.half * NC : 0;
+  const uint32_t colA = PHASE == 1 ? j0 : x.half * 128;
+  const uint32_t colB = PHASE == 1 ? 128 + j0 : x.half * 128 + NC;
+  const uint32_t tabA = smem_u32(&sm.xs_tab[0][j0]);
+  const uint32_t tabB = smem_u32(&sm.xs_tab[0][PHASE == 1 ? j0 : NC]);
+  const float* swA;
+  const float* swB;
+  if (PHASE == 1) {
+    swA = a.s_gate + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
+    swB = a.s_up + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
+  } else {
+    swA = a.s_down + static_cast<size_t>(tl.g * KBd + tl.n * 2 + x.half) * KBi;
+    swB = swA;
+  }
+  float acc[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) acc[i] = 0.0f;
+  for (int kb = 0; kb < x.KB; ++kb) {
+    const float wA = __ldg(swA + kb), wB = __ldg(swB + kb);
+    if (!warp_wait(&sm.tfull[buf], tphase, x.abort)) return false;
+    tc_fence_after();
+    const uint32_t tb = x.tq + buf * BN;
+    const uint32_t ta = tabA + kb * (NMAX * 4), tt = tabB + kb * (NMAX * 4);
+    if (NC < 32) {
+      // both ranges in flight at once
+      uint32_t r[NV];
+#pragma unroll
+      for (int p = 0; p < NC / 8; ++p) {
+        tmem_ld8_async(tb + colA + 8 * p, &r[8 * p]);
+        tmem_ld8_async(tb + colB + 8 * p, &r[NC + 8 * p]);
+      }
+      tmem_wait_ld(r);
+      tc_fence_before();
+      __syncwarp();
+      if (x.lane == 0) mbar_arrive(&sm.tempty[buf]);
+#pragma unroll
+      for (int p = 0; p < NC / 4; ++p) {
+        const float4 t4 = lds_f4(ta + 16 * p);
+        fma4(&acc[4 * p], t4, wA, &r[4 * p]);
+        fma4(&acc[NC + 4 * p], PHASE == 1 ? t4 : lds_f4(tt + 16 * p), wB, &r[NC + 4 * p]);
+      }
+    } else {
+      // one range at a time, so that 64 accumulators and the loaded values
+      // stay within the register budget
+      uint32_t r[NC];
+#pragma unroll
+      for (int p = 0; p < NC / 8; ++p) tmem_ld8_async(tb + colA + 8 * p, &r[8 * p]);
+      tmem_wait_ld(r);
+#pragma unroll
+      for (int p = 0; p < NC / 4; ++p) fma4(&acc[4 * p], lds_f4(ta + 16 * p), wA, &r[4 * p]);
+#pragma unroll
+      for (int p = 0; p < NC / 8; ++p) tmem_ld8_async(tb + colB + 8 * p, &r[8 * p]);
+      tmem_wait_ld(r);
+      tc_fence_before();
+      __syncwarp();
+      if (x.lane == 0) mbar_arrive(&sm.tempty[buf]);
+#pragma unroll
+      for (int p = 0; p < NC / 4; ++p) fma4(&acc[NC + 4 * p], lds_f4(tt + 16 * p), wB, &r[4 * p]);
+    }
+    buf ^= 1;
+    if (buf == 0) tphase ^= 1;
+  }
+  __syncwarp();
+  if (x.lane == 0) mbar_arrive(&sm.dbar);   // this warp no longer reads the table
+
+  const int c = x.q * 32 + x.lane;           // weight row within the 128-row tile
+  if (PHASE == 1) {
+    float hv[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) hv[i] = silu_fast(acc[i]) * acc[NC + i];
+    float* am = &sm.amax_x[xpar][0][0];      // [lane quadrant][token]
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      float m = fabsf(hv[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (x.lane == 0) am[x.q * NMAX + j0 + i] = m;
+    }
+    __syncwarp();
+    if (x.lane == 0) mbar_arrive(&sm.xbar);
+    if (!warp_wait(&sm.xbar, xpar, x.abort)) return false;
+    xpar ^= 1;
+    const size_t col = static_cast<size_t>(tl.n) * 128 + c;
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const int tok = j0 + i;
+      const float m = fmaxf(fmaxf(am[tok], am[NMAX + tok]), fmaxf(am[2 * NMAX + tok], am[3 * NMAX + tok]));
+      const float sc = tile_scale(m);
+      if (tok < tl.mrows) {
+        // H rows: routed rows as in xq_perm, then the shared expert's T rows
+        const size_t hrow = static_cast<size_t>((tl.shared ? a.P : 0) + r0 + tok);
+        // the scale follows the stored rule; the code multiplies by its reciprocal
+        a.H[hrow * a.I + col] = static_cast<uint8_t>(e4m3x2(hv[i] * __fdiv_rn(1.0f, sc), 0.0f) & 0xFF);
+        if (c == 0) a.Hs[hrow * KBi + tl.n] = sc;
+      }
+    }
+  } else {
+    // output channel n*256 + half*128 + c of each token: a warp writes 32
+    // consecutive channels (128 bytes) of one token at a time
+    float* y = (tl.shared ? a.y_shared + static_cast<size_t>(r0 - a.P) * a.d
+                          : a.y_perm + static_cast<size_t>(r0) * a.d) +
+               (tl.n * BN + x.half * 128 + c);
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      if (j < tl.mrows) y[static_cast<size_t>(j) * a.d] = acc[j];
+  }
+  return true;
+}
+
 template <int PHASE>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_x,
@@ -181,7 +373,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = tiles + STAGES * STAGE_BYTES;   // 1024-aligned (phase 2 only)
-  Smem<STAGES>& sm = *reinterpret_cast<Smem<STAGES>*>(staging + Cfg<PHASE>::STAGING);
+  using SmemT = Smem<STAGES, Cfg<PHASE>::TAB_KB>;
+  SmemT& sm = *reinterpret_cast<SmemT*>(staging + Cfg<PHASE>::STAGING);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
@@ -201,6 +394,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.xbar, EPI_WARPS);
+    mbar_init(&sm.sbar, EPI_WARPS);
+    mbar_init(&sm.dbar, EPI_WARPS);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -218,8 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   for (int g = threadIdx.x; g < G; g += THREADS) {
     const int rows = g == a.N_r ? a.T : sm.off[g + 1] - sm.off[g];
-    const int wide = rows - narrow_part(rows, a.narrow_max);
-    sm.tile_start[g] = ((wide + BM - 1) / BM) * n_tiles;
+    sm.tile_start[g] = ((rows + BM - 1) / BM) * n_tiles;
   }
   __syncthreads();
   if (warp == 0) {  // exclusive prefix sum of tile counts, in place
@@ -295,16 +489,34 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t tphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
+        // narrow tile: the weights are M (two 128-row MMAs into columns 0 and
+        // 128 of the buffer), the tile's first N = rows rounded up to 16 token
+        // rows of the A stage are N
+        const uint32_t idesc_n = make_idesc(0, 0, 128, (tl.mrows + 15) & ~15);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) { ok = false; break; }
           if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
           const uint64_t ad = sw128_kmajor_desc(a_addr);
-          const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
           const uint32_t d_tmem = tmem + buf * BN;
+          if (!tl.narrow) {
+            const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 32; ++k) umma_f8f6f4(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0);
+            for (int k = 0; k < BK / 32; ++k) umma_f8f6f4(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0);
+          } else {
+            // the two accumulators' K steps interleaved: an MMA costs about
+            // the same for N <= 64 as for N = 256, and two independent chains
+            // overlap in the tensor pipe where one dependent chain does not
+            const uint64_t wd0 = sw128_kmajor_desc(a_addr + A_BYTES);
+            const uint64_t wd1 = sw128_kmajor_desc(a_addr + A_BYTES + B_BYTES / 2);
+#pragma unroll
+            for (int k = 0; k < BK / 32; ++k) {
+              umma_f8f6f4(d_tmem, wd0 + 2 * k, ad + 2 * k, idesc_n, k > 0);
+              umma_f8f6f4(d_tmem + 128, wd1 + 2 * k, ad + 2 * k, idesc_n, k > 0);
+            }
+          }
           umma_commit(&sm.empty[stage]);
           umma_commit(&sm.tfull[buf]);
           if (++stage == STAGES) {
@@ -330,9 +542,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     int buf = 0;
     uint32_t tphase = 0;
     uint32_t xpar = 0;
+    int n_narrow = 0;     // narrow tiles done (parity of sbar / dbar)
     const int KBd = a.d / BK, KBi = a.I / BK;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
+      if (tl.narrow) {
+        NarrowCtx c{tmem + lane_base, q, half, lane, ew * 32 + lane, KB, abort};
+        bool ok = false;
+        switch ((tl.mrows + 15) >> 4) {   // N = 16, 32, 48 or 64
+          case 1: ok = narrow_tile<PHASE, 8>(sm, a, tl, c, buf, tphase, xpar, n_narrow); break;
+          case 2: ok = narrow_tile<PHASE, 16>(sm, a, tl, c, buf, tphase, xpar, n_narrow); break;
+          case 3: ok = narrow_tile<PHASE, 24>(sm, a, tl, c, buf, tphase, xpar, n_narrow); break;
+          default: ok = narrow_tile<PHASE, 32>(sm, a, tl, c, buf, tphase, xpar, n_narrow); break;
+        }
+        if (!ok) break;
+        continue;
+      }
       const int rr = tl.m * BM + r;          // row within the group
       const bool valid = rr < tl.rows;
       const int grow = tl.row0 + rr;         // row in the A tensor (and its scales)
@@ -498,8 +723,6 @@ inline int make_tmap_y(CUtensorMap* m, const float* base, uint64_t rows, uint64_
 }  // namespace gg
 }  // namespace moe
 
-#include "gemm_narrow.cu"
-
 extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
   (void)d;
   if (T <= 0 || K_r <= 0 || I <= 0) return 0;
@@ -507,12 +730,15 @@ extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
   return moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float);
 }
 
-// the narrow kernels need the tile's K-block factor table to fit shared memory
-static bool narrow_enabled(int d, int I) { return d / moe::gg::BK <= moe::gn::MAX_KB && I / moe::gg::BK <= moe::gn::MAX_KB; }
+// narrow tiles need the tile's [kb][token] activation-scale table to fit
+// shared memory
+static bool narrow_enabled(int d, int I) {
+  return d / moe::gg::BK <= moe::gg::MAX_KB_N1 && I / moe::gg::BK <= moe::gg::MAX_KB_N2;
+}
 
 extern "C" int moe_grouped_gemm_fp8_launches(int d, int I) {
   if (d <= 0 || I <= 0) return -1;
-  return narrow_enabled(d, I) ? 4 : 2;
+  return 2;
 }
 
 extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
@@ -551,15 +777,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
   if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
   if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
-  // narrow tiles: token operands in boxes of 64 rows, W_down in 128-row boxes
   const bool narrow = narrow_enabled(d, I);
-  CUtensorMap tnX, tnXs, tnH, tnWd;
-  if (narrow) {
-    if (int st = make_tmap_2d(&tnX, xq_perm, U8, 1, P, d, gn::NMAX, BK)) return st;
-    if (int st = make_tmap_2d(&tnXs, xq, U8, 1, T, d, gn::NMAX, BK)) return st;
-    if (int st = make_tmap_2d(&tnH, H, U8, 1, rowsH, I, gn::NMAX, BK)) return st;
-    if (int st = make_tmap_2d(&tnWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, 128, BK)) return st;
-  }
 
   Args args;
   args.offsets = offsets;
@@ -577,7 +795,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   args.Hs = Hs;
   args.y_perm = y_perm;
   args.y_shared = y_shared;
-  args.narrow_max = narrow ? gn::NMAX : 0;
+  args.narrow_max = narrow ? NMAX : 0;
 
   // upper bound on row tiles: every non-empty routed group wastes < 1 tile
   const long long m_tiles = (P + BM - 1) / BM + (P < N_r ? P : N_r) + (T + BM - 1) / BM;
@@ -594,30 +812,9 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
                            "smem attribute (down)"))
     return st;
-  // narrow tiles: at most one per group and column tile
-  const int gn1 = std::min<long long>(di.sm_count, static_cast<long long>(N_r + 1) * (I / 128));
-  const int gn2 = std::min<long long>(di.sm_count, static_cast<long long>(N_r + 1) * (d / 256));
-  auto n1 = gn::narrow_gemm_kernel<1>;
-  auto n2 = gn::narrow_gemm_kernel<2>;
-  if (narrow) {
-    if (int st = cuda_status(cudaFuncSetAttribute(n1, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   static_cast<int>(gn::SMEM_BYTES)), "smem attribute (narrow gate/up)"))
-      return st;
-    if (int st = cuda_status(cudaFuncSetAttribute(n2, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   static_cast<int>(gn::SMEM_BYTES)), "smem attribute (narrow down)"))
-      return st;
-  }
   k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
-  if (narrow) {
-    n1<<<gn1, gn::THREADS, gn::SMEM_BYTES, s>>>(tnX, tnXs, tmWg, tmWu, args);
-    if (int st = launch_status("narrow GEMM launch (gate/up)")) return st;
-  }
   k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (down)")) return st;
-  if (narrow) {
-    n2<<<gn2, gn::THREADS, gn::SMEM_BYTES, s>>>(tnH, tnH, tnWd, tnWd, args);
-    if (int st = launch_status("narrow GEMM launch (down)")) return st;
-  }
   return MOE_OK;
 }

@@ -186,10 +186,9 @@ MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
 
 /*
  * moe_grouped_gemm_fp8_launches: number of kernel launches one
- * moe_grouped_gemm_fp8 call with these sizes makes on its stream (2, or 4
- * when the narrow-tile kernels for groups of at most 64 rows are enabled:
- * d/128 <= 56 and I/128 <= 56). A host-side query; no device work. The
- * pages have no counterpart: it exists so that callers can account for
+ * moe_grouped_gemm_fp8 call with these sizes makes on its stream (2: the
+ * gate/up launch and the down launch). A host-side query; no device work.
+ * The pages have no counterpart: it exists so that callers can account for
  * launches. Returns -1 for non-positive sizes.
  */
 MOE_API int moe_grouped_gemm_fp8_launches(int d, int I);

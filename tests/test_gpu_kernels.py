@@ -234,6 +234,10 @@ def _gemm_case(d, I, counts, T, seed):
     (512, 256, [3, 0, 128, 64, 200], 129),
     (2048, 1024, [384, 200], 256),
     (7168, 2048, [5, 300], 130),
+    # groups of at most 64 rows run as narrow tiles: every token-width class
+    # (N = 16, 32, 48, 64) and its edges, next to wide groups; T = 40 makes
+    # the shared expert narrow too
+    (512, 256, [16, 17, 33, 48, 49, 63, 64, 65, 0, 1], 40),
 ])
 def test_grouped_gemm_fp8(lib, d, I, counts, T):
     from fine_grained_fp8_sigmoid_b200 import binding as B
