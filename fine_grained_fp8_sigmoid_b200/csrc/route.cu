@@ -15,9 +15,22 @@
 // K block (the read-back competes with the MMAs for TMEM).
 // After the K loop the logits are parked in the (now idle) pipeline shared
 // memory, so sigmoid and the top-K insertion run as a compact rolled loop.
+//
+// Split K: with few token tiles (decode: one), a single CTA per tile would
+// stream all of d through one SM. The launch then forms clusters of S CTAs
+// per tile (S a power of two <= 8, S * tiles <= SMs); CTA rank r of the
+// cluster runs its share of the K groups and parks its FP32 partial logits,
+// and after a cluster barrier rank 0 adds the other ranks' partials, in rank
+// order, through distributed shared memory before the sigmoid and top-K. A
+// second cluster barrier keeps every rank's shared memory alive until rank 0
+// has read it.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
 // epilogue (TMEM lane quadrant w%4, column half (w-4)/4), which finishes
 // with sigmoid, the biased top-K of each half, and a merge of the halves.
+// The top-K of a half runs as several independent insertion lists over
+// consecutive column blocks (their compare-and-shift chains interleave),
+// merged in block order; the selected experts' affinities are recomputed
+// from the parked logits for the gates.
 #include "host.cuh"
 
 namespace moe {
@@ -87,7 +100,27 @@ __device__ __forceinline__ void topk_store(const int (&ii)[KMAX], const float (&
   }
 }
 
-__device__ __forceinline__ float sigmoidf(float z) { return __fdiv_rn(1.0f, 1.0f + expf(-z)); }
+// sigmoid with the hardware exponential and reciprocal (relative error
+// ~1e-6, far inside the routing acceptance margin); sigmoid(0) = 0.5 exactly
+__device__ __forceinline__ float sigmoid_fast(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+
+// top-K of (key, index) pairs, keys descending; strict comparison, so an
+// equal key inserted later (a higher index) stays behind
+template <int KMAX>
+__device__ __forceinline__ void topk_insert_ki(float (&kk)[KMAX], int (&ii)[KMAX], float key, int idx) {
+  bool shifting = false;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const bool take = shifting || (key > kk[j]);
+    const float tk = kk[j];
+    const int ti = ii[j];
+    kk[j] = take ? key : tk;
+    ii[j] = take ? idx : ti;
+    key = take ? tk : key;
+    idx = take ? ti : idx;
+    shifting = take;
+  }
+}
 
 template <int KMAX>
 struct Smem {
@@ -102,7 +135,6 @@ struct Smem {
   float bias[NP];
   float m_key[KMAX][BM];   // top-K of the upper column half, handed to the lower half
   int m_idx[KMAX][BM];
-  float m_s[KMAX][BM];
 };
 
 template <int KMAX>
@@ -110,10 +142,34 @@ constexpr size_t router_smem_bytes() {
   return 1024 + STAGES * STAGE_BYTES + sizeof(Smem<KMAX>);
 }
 
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Eight FP32 at local[0], local[BM], ..., local[7 * BM] of CTA `rank` of the
+// cluster (the same shared-memory offsets there), eight loads in flight.
+__device__ __forceinline__ void ld_cluster_f32x8(const float* local, uint32_t rank, float (&v)[8]) {
+  static_assert(BM * 4 == 512, "row stride of the parked logits");
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile(
+      "ld.shared::cluster.f32 %0, [%8];\n\t"
+      "ld.shared::cluster.f32 %1, [%8+512];\n\t"
+      "ld.shared::cluster.f32 %2, [%8+1024];\n\t"
+      "ld.shared::cluster.f32 %3, [%8+1536];\n\t"
+      "ld.shared::cluster.f32 %4, [%8+2048];\n\t"
+      "ld.shared::cluster.f32 %5, [%8+2560];\n\t"
+      "ld.shared::cluster.f32 %6, [%8+3072];\n\t"
+      "ld.shared::cluster.f32 %7, [%8+3584];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+      : "r"(remote)
+      : "memory");
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(THREADS, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_e,
-                  const float* __restrict__ b, int T, int d, int N_r, int K,
+                  const float* __restrict__ b, int T, int d, int N_r, int K, int S,
                   float* __restrict__ scores_out, int32_t* __restrict__ topk_idx,
                   float* __restrict__ gates) {
   extern __shared__ uint8_t smem_raw[];
@@ -123,8 +179,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  const int tile = blockIdx.x;
+  const int tile = blockIdx.x / S;
+  const int rank = blockIdx.x % S;          // rank in the cluster of S CTAs (1-D clusters)
   const int KB = d / BK;
+  // this rank's K blocks: whole partial groups of RK blocks
+  const int NG_all = (KB + RK - 1) / RK;
+  const int g_lo = rank * NG_all / S, g_hi = (rank + 1) * NG_all / S;
+  const int kb_lo = g_lo * RK, kb_hi = min(g_hi * RK, KB);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -161,9 +222,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // producer: K blocks of u (128 x 64) and e (256 x 64, rows >= N_r read as zero)
       int armed[STAGES];
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        const int s = (kb - kb_lo) % STAGES;
+        const uint32_t ph = ((kb - kb_lo) / STAGES) & 1;
         if (!mbar_wait(&sm.empty[s], ph ^ 1, abort)) break;
         uint8_t* a_dst = tiles + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&sm.full[s], STAGE_BYTES);
@@ -179,10 +240,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     } else if (warp == 1 && lane == 0) {
       const uint32_t idesc = make_idesc(1, 1, BM, NP);
-      for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        const int grp = kb / RK;                 // partial buffer group
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        const int s = (kb - kb_lo) % STAGES;
+        const uint32_t ph = ((kb - kb_lo) / STAGES) & 1;
+        const int grp = kb / RK - g_lo;          // partial buffer group of this rank
         const int buf = grp & 1;
         const bool first = kb % RK == 0, last = kb % RK == RK - 1 || kb == KB - 1;
         if (first && !mbar_wait(&sm.tempty[buf], ((grp >> 1) & 1) ^ 1, abort)) break;
@@ -213,7 +274,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
     bool ok = true;
-    const int NG = (KB + RK - 1) / RK;
+    const int NG = g_hi - g_lo;
     for (int grp = 0; grp < NG; ++grp) {
       const int buf = grp & 1;
       if (!warp_wait(&sm.tfull[buf], (grp >> 1) & 1, abort)) { ok = false; break; }
@@ -229,45 +290,116 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tempty[buf]);
     }
-    if (ok) {
-      // Every TMA load was consumed by an MMA and every MMA has completed
-      // (the last partial has been read), so the stage buffers are free:
-      // park this thread's 128 logits there, column-major so that a warp's
-      // accesses fall in consecutive banks, and walk them in a rolled loop.
-      float* park = reinterpret_cast<float*>(tiles) + half * 128 * BM;
+    // Every TMA load was consumed by an MMA and every MMA has completed (the
+    // last partial has been read), so the stage buffers are free: park this
+    // thread's 128 logits there, column-major so that a warp's accesses fall
+    // in consecutive banks, and walk them in a rolled loop.
+    float* park = reinterpret_cast<float*>(tiles) + half * 128 * BM;
+    if (ok && S > 1 && rank > 0) {
 #pragma unroll
       for (int j = 0; j < 128; ++j) park[j * BM + r] = acc[j];
-      float kk[KMAX], ss[KMAX];
-      int ii[KMAX];
-      topk_init(kk, ii, ss);
+    }
+    if (S > 1) {
+      cluster_sync_all();     // every rank's partial is parked
+      if (ok && rank == 0) {
+        for (int q2 = 1; q2 < S; ++q2) {
+#pragma unroll
+          for (int jb = 0; jb < 16; jb += 4) {   // 32 loads in flight
+            float v[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) ld_cluster_f32x8(park + (jb + u) * 8 * BM + r, q2, v[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc[(jb + u) * 8 + i] += v[u][i];
+          }
+        }
+      }
+    }
+    if (ok && rank == 0) {
+#pragma unroll
+      for (int j = 0; j < 128; ++j) park[j * BM + r] = acc[j];
+      // SUB independent insertion chains over consecutive column blocks (the
+      // chain of compare-and-shift steps, not the arithmetic, bounds a single
+      // list), merged in block order: every index of block c exceeds those of
+      // the blocks before it, so strict-greater insertion keeps equal keys
+      // lowest-index first
+      constexpr int SUB = KMAX == 8 ? 4 : 2;
+      constexpr int LEN = 128 / SUB;
+      float kk[SUB][KMAX];
+      int ii[SUB][KMAX];
+#pragma unroll
+      for (int c = 0; c < SUB; ++c)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+          kk[c][j] = -INFINITY;
+          ii[c][j] = 0x7fffffff;
+        }
       const int ncol = min(128, N_r - half * 128);
       float* srow = (scores_out != nullptr && t < T) ? scores_out + static_cast<size_t>(t) * N_r + half * 128 : nullptr;
+      if (ncol == 128 && srow == nullptr) {
+        // all columns live: no guards, so the chains' instructions interleave
 #pragma unroll 1
-      for (int j = 0; j < ncol; ++j) {
-        const int col = half * 128 + j;
-        const float sg = sigmoidf(park[j * BM + r]);
-        topk_insert(kk, ii, ss, sg + sm.bias[col], col, sg);
-        if (srow != nullptr) srow[j] = sg;
+        for (int j = 0; j < LEN; ++j) {
+          float key[SUB];
+#pragma unroll
+          for (int c = 0; c < SUB; ++c) key[c] = sigmoid_fast(park[(c * LEN + j) * BM + r]) + sm.bias[half * 128 + c * LEN + j];
+#pragma unroll
+          for (int c = 0; c < SUB; ++c) topk_insert_ki(kk[c], ii[c], key[c], half * 128 + c * LEN + j);
+        }
+      } else {
+#pragma unroll 1
+        for (int j = 0; j < LEN; ++j) {
+#pragma unroll
+          for (int c = 0; c < SUB; ++c) {
+            const int jl = c * LEN + j;
+            if (jl < ncol) {
+              const int col = half * 128 + jl;
+              const float sg = sigmoid_fast(park[jl * BM + r]);
+              topk_insert_ki(kk[c], ii[c], sg + sm.bias[col], col);
+              if (srow != nullptr) srow[jl] = sg;
+            }
+          }
+        }
       }
+#pragma unroll
+      for (int c = 1; c < SUB; ++c)
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (ii[c][j] < N_r) topk_insert_ki(kk[0], ii[0], kk[c][j], ii[c][j]);
+      float (&kk0)[KMAX] = kk[0];
+      int (&ii0)[KMAX] = ii[0];
       // the upper half hands its list to the lower half, which merges: every
       // upper-half index exceeds every lower-half one, and the list arrives
       // in (key desc, index asc) order, so equal keys stay lowest-index first
       if (half == 1) {
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-          sm.m_key[j][r] = kk[j];
-          sm.m_idx[j][r] = ii[j];
-          sm.m_s[j][r] = ss[j];
+          sm.m_key[j][r] = kk0[j];
+          sm.m_idx[j][r] = ii0[j];
         }
       }
       mbar_arrive(&sm.xbar);
       if (half == 0 && warp_wait(&sm.xbar, 0, abort)) {
 #pragma unroll
         for (int j = 0; j < KMAX; ++j)
-          if (sm.m_idx[j][r] < N_r) topk_insert(kk, ii, ss, sm.m_key[j][r], sm.m_idx[j][r], sm.m_s[j][r]);
-        if (t < T) topk_store(ii, ss, K, topk_idx + static_cast<size_t>(t) * K, gates + static_cast<size_t>(t) * K);
+          if (sm.m_idx[j][r] < N_r) topk_insert_ki(kk0, ii0, sm.m_key[j][r], sm.m_idx[j][r]);
+        // the affinities of the selected experts, recomputed from the parked
+        // logits ([expert][token], both halves) exactly as for their keys
+        const float* logits = reinterpret_cast<const float*>(tiles);
+        float ss0[KMAX];
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) ss0[j] = ii0[j] < N_r ? sigmoid_fast(logits[ii0[j] * BM + r]) : 0.0f;
+        if (t < T) topk_store(ii0, ss0, K, topk_idx + static_cast<size_t>(t) * K, gates + static_cast<size_t>(t) * K);
       }
     }
+  }
+  if (S > 1) {
+    // the control warps meet the epilogue's first barrier here; the second
+    // keeps every rank's parked partial alive until rank 0 has read it
+    __syncwarp();
+    if (warp < EPI_WARP0) cluster_sync_all();
+    cluster_sync_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -329,21 +461,35 @@ extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
   CUtensorMap tm_u, tm_e;
   if (int st = make_tmap_2d(&tm_u, u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, d, BM, BK)) return st;
   if (int st = make_tmap_2d(&tm_e, e, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N_r, d, NP, BK)) return st;
-  const int blocks = (T + BM - 1) / BM;
-  if (K_r <= 8) {
-    auto k = router_kernel<8>;
-    constexpr size_t smem = router_smem_bytes<8>();
-    if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
-                             "router smem attribute"))
-      return st;
-    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, K_r, scores_out, topk_idx, gates);
-  } else {
-    auto k = router_kernel<16>;
-    constexpr size_t smem = router_smem_bytes<16>();
-    if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
-                             "router smem attribute"))
-      return st;
-    k<<<blocks, THREADS, smem, s>>>(tm_u, tm_e, b, T, d, N_r, K_r, scores_out, topk_idx, gates);
+  const int tiles = (T + BM - 1) / BM;
+  const int NG_all = (d / BK + RK - 1) / RK;
+  auto k = K_r <= 8 ? router_kernel<8> : router_kernel<16>;
+  const size_t smem = K_r <= 8 ? router_smem_bytes<8>() : router_smem_bytes<16>();
+  if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                           "router smem attribute"))
+    return st;
+  // split K over a cluster of S CTAs per token tile while the SMs allow
+  int S = 1;
+  while (S < 8 && tiles * S * 2 <= di.sm_count && S * 2 <= NG_all) S *= 2;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  for (;; S /= 2) {   // a cluster size the device can place
+    cfg.gridDim = dim3(tiles * S);
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    int n_clusters = 0;
+    if (S == 1 || (cudaOccupancyMaxActiveClusters(&n_clusters, k, &cfg) == cudaSuccess && n_clusters > 0)) break;
+    cudaGetLastError();
   }
+  if (int st = cuda_status(cudaLaunchKernelEx(&cfg, k, tm_u, tm_e, b, T, d, N_r, K_r, S, scores_out, topk_idx, gates),
+                           "router launch"))
+    return st;
   return launch_status();
 }

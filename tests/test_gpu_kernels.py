@@ -116,7 +116,7 @@ def _check_routing(gpu_idx, s64, b, K, margin=1e-5):
     return diff
 
 
-@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", None), ("mid", 1000), ("prefill", 1500),
+@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", None), ("mid", 1000), ("mid", 5000), ("prefill", 1500),
                                     ("decode", None)])
 def test_router_tensor_cores(lib, name, T):
     from fine_grained_fp8_sigmoid_b200 import binding as B
