@@ -777,7 +777,13 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
   if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
   if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
-  const bool narrow = narrow_enabled(d, I);
+  // Narrow tiles only when the average routed group has at most 64 rows
+  // (decode-like batches). With larger groups the few small ones gain little
+  // (an N <= 64 MMA costs about as much as an N = 256 one) and their slower
+  // tiles put the CTAs of the round-robin schedule out of step, so that tiles
+  // sharing weights and activation rows no longer meet in L2 (measured at
+  // T = 8192 with 39 groups of <= 64 rows: +4.2 GB of DRAM reads).
+  const bool narrow = narrow_enabled(d, I) && P <= static_cast<long long>(NMAX) * N_r;
 
   Args args;
   args.offsets = offsets;
