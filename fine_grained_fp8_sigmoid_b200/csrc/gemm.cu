@@ -699,10 +699,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
         }
       }
-      // END_OF_EPILOGUE_TILE
     }
-    if (PHASE == 2 && lane == 0) bulk_wait_all();
-    // END_OF_EPILOGUE
+    if (PHASE == 2 && lane == 0) bulk_wait_all();   // outputs written before the CTA exits
   }
 
   tc_fence_before();
