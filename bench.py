@@ -102,6 +102,19 @@ def weight_bytes(cfg):
     return (cfg.N_r + 1) * per
 
 
+def gemm_algorithmic_bytes(cfg, touched_routed):
+    """Bytes one moe_grouped_gemm_fp8 call must move at least: the weights of
+    the touched routed experts and the shared one, read once; the permuted
+    and shared activations with their scales; the intermediate H written and
+    read back; the FP32 outputs written."""
+    per_expert = 3 * cfg.d * cfg.I + 3 * (cfg.d // 128) * (cfg.I // 128) * 4
+    rows = cfg.T * cfg.K_r + cfg.T
+    acts = rows * (cfg.d + cfg.d // 128 * 4)
+    inter = 2 * rows * (cfg.I + cfg.I // 128 * 4)
+    outs = rows * cfg.d * 4
+    return (touched_routed + 1) * per_expert + acts + inter + outs
+
+
 def workload_desc(cfg):
     return (f"DeepSeek-V3 MoE layer, {cfg.name}: T={cfg.T}, d={cfg.d}, {cfg.N_r} routed experts "
             f"top-{cfg.K_r} + 1 shared, SwiGLU I={cfg.I}, E4M3 1x128/128x128 scales")
@@ -283,9 +296,26 @@ def run_ours(args, rank, world, local_rank):
 
     flops = layer_flops(cfg)
     gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
-    fp8_peak = 2.0 * peaks["bf16"]          # dense FP8 = 2x dense BF16 (nominal ratio)
+    # dense FP8 = 2x dense BF16 (nominal ratio). The GEMM is timed inside a
+    # long run of back-to-back steps under the power cap, so the sustained
+    # figure is its denominator; the burst one is reported beside it.
+    fp8_peak = 2.0 * peaks["bf16_sustained"]
+    fp8_burst = 2.0 * peaks["bf16"]
     achieved_tf = flops / gemm_avg_s / 1e12
     layer_tf = flops / (ms_step / 1e3) / 1e12
+    touched = int((layer.counts > 0).sum().item())
+    gemm_bytes = gemm_algorithmic_bytes(cfg, touched)
+    achieved_gbs = gemm_bytes / gemm_avg_s / 1e9
+    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)      # FLOP per byte
+    if flops / gemm_bytes >= ridge:
+        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
+                "frac": achieved_tf / fp8_peak,
+                "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TF/s x2",
+                "frac_of_burst": achieved_tf / fp8_burst}
+    else:
+        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved_gbs / peaks["hbm_gbs"],
+                "peak_source": f"{peaks['source']} copy bandwidth {peaks['hbm_gbs']} GB/s"}
 
     balance = None
     if cfg.name == "skew":
@@ -346,11 +376,10 @@ def run_ours(args, rank, world, local_rank):
                              "weights stream every step"},
             "tflops": layer_tf,
             "pct_fp8_peak": layer_tf / fp8_peak,
-            "roofline": {"bound": "tensor", "kernel": f"moe_grouped_gemm_fp8 ({gemm_launches} launches)",
-                         "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": achieved_tf / fp8_peak, "traffic": gemm_traffic(cfg),
-                         "peak_source": f"{peaks['source']} bf16 {peaks['bf16']} TF/s x2 (burst)",
-                         "gemm_ms": float(np.mean(gemm_ms))},
+            "roofline": dict(roof, kernel=f"moe_grouped_gemm_fp8 ({gemm_launches} launches)",
+                             traffic=gemm_traffic(cfg), gemm_ms=float(np.mean(gemm_ms)),
+                             gemm_tflops=achieved_tf, algorithmic_bytes=gemm_bytes,
+                             experts_touched=touched + 1),
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_tps, "unit": "tokens/s",
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2},
