@@ -14,29 +14,27 @@
 // FP32 rounding while reading the 128 x 256 partial back only every fourth
 // K block (the read-back competes with the MMAs for TMEM).
 // After the K loop the logits are parked in the (now idle) pipeline shared
-// memory, so sigmoid and the top-K insertion run as a compact rolled loop.
+// memory as [expert][token].
 //
 // Split K: with few token tiles (decode: one), a single CTA per tile would
 // stream all of d through one SM. The launch then forms clusters of S CTAs
 // per tile (S a power of two <= 8, S * tiles <= SMs); CTA rank r of the
-// cluster runs its share of the K groups and parks its FP32 partial logits,
-// and after a cluster barrier rank 0 adds the other ranks' partials, in rank
-// order, through distributed shared memory before the sigmoid and top-K. A
-// second cluster barrier keeps every rank's shared memory alive until rank 0
-// has read it.
+// cluster runs its share of the K groups and parks its FP32 partial logits.
+// After a cluster barrier every rank takes 128/S of the tile's tokens: a
+// token's experts are spread over 2S threads of consecutive lanes, each adds
+// the ranks' partials in rank order through distributed shared memory
+// (deterministic), forms the affinity and biased key and keeps a top-K list,
+// and the 2S lists merge by shuffles. A second cluster barrier keeps every
+// rank's shared memory alive until all ranks have read it.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
-// epilogue (TMEM lane quadrant w%4, column half (w-4)/4), which finishes
-// with sigmoid, the biased top-K of each half, and a merge of the halves.
-// The top-K of a half runs as several independent insertion lists over
-// consecutive column blocks (their compare-and-shift chains interleave),
-// merged in block order; the selected experts' affinities are recomputed
-// from the parked logits for the gates.
+// epilogue (TMEM lane quadrant w%4, column half (w-4)/4 while reading TMEM).
 #include "host.cuh"
 
 namespace moe {
 namespace route {
 
 constexpr int BM = 128;          // tokens per CTA (TMEM lanes)
+constexpr int PR = 260;          // parked logits: floats per token row (256 experts + 4 pad, 16-byte rows)
 constexpr int BK = 64;           // bf16 per K block = 128 bytes = one swizzle row
 constexpr int NP = 256;          // MMA N: all experts of a token in one tile
 constexpr int STAGES = 4;
@@ -129,13 +127,12 @@ struct Smem {
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
-  uint64_t xbar;
   uint32_t tmem_base;
   int abort;
   float bias[NP];
-  float m_key[KMAX][BM];   // top-K of the upper column half, handed to the lower half
-  int m_idx[KMAX][BM];
 };
+
+static_assert(BM * PR * 4 <= STAGES * STAGE_BYTES, "parked logits fit the pipeline stages");
 
 template <int KMAX>
 constexpr size_t router_smem_bytes() {
@@ -146,24 +143,45 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Eight FP32 at local[0], local[BM], ..., local[7 * BM] of CTA `rank` of the
-// cluster (the same shared-memory offsets there), eight loads in flight.
-__device__ __forceinline__ void ld_cluster_f32x8(const float* local, uint32_t rank, float (&v)[8]) {
-  static_assert(BM * 4 == 512, "row stride of the parked logits");
+// FP32 at byte offset `off` from `base` (a shared-memory address of this
+// CTA) in CTA `rank` of the cluster
+__device__ __forceinline__ float ld_cluster_f32(uint32_t base, uint32_t rank) {
   uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(base), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// Two float4 at base + off0 and base + off1 in CTA `rank` of the cluster
+__device__ __forceinline__ void ld_cluster_f32x4x2(uint32_t base, uint32_t off0, uint32_t off1, uint32_t rank,
+                                                   float (&v)[8]) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(base), "r"(rank));
   asm volatile(
-      "ld.shared::cluster.f32 %0, [%8];\n\t"
-      "ld.shared::cluster.f32 %1, [%8+512];\n\t"
-      "ld.shared::cluster.f32 %2, [%8+1024];\n\t"
-      "ld.shared::cluster.f32 %3, [%8+1536];\n\t"
-      "ld.shared::cluster.f32 %4, [%8+2048];\n\t"
-      "ld.shared::cluster.f32 %5, [%8+2560];\n\t"
-      "ld.shared::cluster.f32 %6, [%8+3072];\n\t"
-      "ld.shared::cluster.f32 %7, [%8+3584];"
+      "ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%8];\n\t"
+      "ld.shared::cluster.v4.f32 {%4, %5, %6, %7}, [%9];"
       : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-      : "r"(remote)
+      : "r"(remote + off0), "r"(remote + off1)
       : "memory");
+}
+
+// Merges one (key, index) into a top-K list ordered by key descending, then
+// index ascending, whatever the order the entries arrive in.
+template <int KMAX>
+__device__ __forceinline__ void topk_insert_lex(float (&kk)[KMAX], int (&ii)[KMAX], float key, int idx) {
+  bool shifting = false;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const bool take = shifting || key > kk[j] || (key == kk[j] && idx < ii[j]);
+    const float tk = kk[j];
+    const int ti = ii[j];
+    kk[j] = take ? key : tk;
+    ii[j] = take ? idx : ti;
+    key = take ? tk : key;
+    idx = take ? ti : idx;
+    shifting = take;
+  }
 }
 
 template <int KMAX>
@@ -197,7 +215,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.tempty[i], EPI_THREADS / 32);
     }
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.xbar, EPI_THREADS);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -268,7 +285,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     const int half = (warp - EPI_WARP0) >> 2;
     const int r = q * 32 + lane;
-    const int t = tile * BM + r;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     float acc[128];
 #pragma unroll
@@ -292,106 +308,103 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // Every TMA load was consumed by an MMA and every MMA has completed (the
     // last partial has been read), so the stage buffers are free: park this
-    // thread's 128 logits there, column-major so that a warp's accesses fall
-    // in consecutive banks, and walk them in a rolled loop.
-    float* park = reinterpret_cast<float*>(tiles) + half * 128 * BM;
-    if (ok && S > 1 && rank > 0) {
+    // CTA's partial logits there as [token][expert] rows of PR floats
+    // (16-byte stores; readers take 16-byte runs of a token's row).
+    float* park = reinterpret_cast<float*>(tiles);
+    if (ok) {
+      float4* row = reinterpret_cast<float4*>(park + r * PR + half * 128);
 #pragma unroll
-      for (int j = 0; j < 128; ++j) park[j * BM + r] = acc[j];
+      for (int m = 0; m < 32; ++m) row[m] = make_float4(acc[4 * m], acc[4 * m + 1], acc[4 * m + 2], acc[4 * m + 3]);
     }
-    if (S > 1) {
-      cluster_sync_all();     // every rank's partial is parked
-      if (ok && rank == 0) {
-        for (int q2 = 1; q2 < S; ++q2) {
+    if (S > 1) cluster_sync_all();           // every rank's partial is parked
+    else named_bar_sync(1, EPI_THREADS);
+
+    // The tile's tokens are split over the S ranks, a token's experts over
+    // TPT = 2S threads in consecutive lanes: thread ch owns the runs of 4
+    // experts 4*(ch + TPT*m), so a warp's 16-byte loads of a token's row are
+    // contiguous. A thread adds the ranks' partials in rank order, forms the
+    // affinity and the biased key, and keeps a top-K list; the TPT lists of a
+    // token then merge in a butterfly of shuffles.
+    const int TPC = BM / S, TPT = EPI_THREADS / TPC, RUNS = NP / (4 * TPT);
+    const int etid = (warp - EPI_WARP0) * 32 + lane;
+    const int rr = rank * TPC + etid / TPT;     // token row in the tile
+    const int ch = etid % TPT;
+    const int tt = tile * BM + rr;
+    float* srow = (scores_out != nullptr && tt < T) ? scores_out + static_cast<size_t>(tt) * N_r : nullptr;
+    const uint32_t tok_base = smem_u32(park + rr * PR);   // this token's row, this CTA
+    // two insertion lists (the two runs of each step), merged at the end
+    float ka[KMAX], kb2[KMAX];
+    int ia[KMAX], ib[KMAX];
 #pragma unroll
-          for (int jb = 0; jb < 16; jb += 4) {   // 32 loads in flight
-            float v[4][8];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) ld_cluster_f32x8(park + (jb + u) * 8 * BM + r, q2, v[u]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int i = 0; i < 8; ++i) acc[(jb + u) * 8 + i] += v[u][i];
-          }
-        }
-      }
+    for (int j = 0; j < KMAX; ++j) {
+      ka[j] = kb2[j] = -INFINITY;
+      ia[j] = ib[j] = 0x7fffffff;
     }
-    if (ok && rank == 0) {
-#pragma unroll
-      for (int j = 0; j < 128; ++j) park[j * BM + r] = acc[j];
-      // SUB independent insertion chains over consecutive column blocks (the
-      // chain of compare-and-shift steps, not the arithmetic, bounds a single
-      // list), merged in block order: every index of block c exceeds those of
-      // the blocks before it, so strict-greater insertion keeps equal keys
-      // lowest-index first
-      constexpr int SUB = KMAX == 8 ? 4 : 2;
-      constexpr int LEN = 128 / SUB;
-      float kk[SUB][KMAX];
-      int ii[SUB][KMAX];
-#pragma unroll
-      for (int c = 0; c < SUB; ++c)
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          kk[c][j] = -INFINITY;
-          ii[c][j] = 0x7fffffff;
-        }
-      const int ncol = min(128, N_r - half * 128);
-      float* srow = (scores_out != nullptr && t < T) ? scores_out + static_cast<size_t>(t) * N_r + half * 128 : nullptr;
-      if (ncol == 128 && srow == nullptr) {
-        // all columns live: no guards, so the chains' instructions interleave
 #pragma unroll 1
-        for (int j = 0; j < LEN; ++j) {
-          float key[SUB];
-#pragma unroll
-          for (int c = 0; c < SUB; ++c) key[c] = sigmoid_fast(park[(c * LEN + j) * BM + r]) + sm.bias[half * 128 + c * LEN + j];
-#pragma unroll
-          for (int c = 0; c < SUB; ++c) topk_insert_ki(kk[c], ii[c], key[c], half * 128 + c * LEN + j);
-        }
+    for (int m = 0; m < RUNS; m += 2) {        // RUNS = 32 / S: 4 (S = 8) .. 32 (S = 1)
+      const int ca = 4 * (ch + TPT * m), cb = 4 * (ch + TPT * (m + 1));
+      if (ca >= N_r) break;                    // every later run starts higher
+      float z[8];
+      if (S == 1) {
+        const float4 a0 = *reinterpret_cast<const float4*>(park + rr * PR + ca);
+        const float4 a1 = *reinterpret_cast<const float4*>(park + rr * PR + cb);
+        z[0] = a0.x; z[1] = a0.y; z[2] = a0.z; z[3] = a0.w;
+        z[4] = a1.x; z[5] = a1.y; z[6] = a1.z; z[7] = a1.w;
       } else {
-#pragma unroll 1
-        for (int j = 0; j < LEN; ++j) {
+        // every rank's values in flight before the sums (in rank order)
+        float v[8][8];
 #pragma unroll
-          for (int c = 0; c < SUB; ++c) {
-            const int jl = c * LEN + j;
-            if (jl < ncol) {
-              const int col = half * 128 + jl;
-              const float sg = sigmoid_fast(park[jl * BM + r]);
-              topk_insert_ki(kk[c], ii[c], sg + sm.bias[col], col);
-              if (srow != nullptr) srow[jl] = sg;
-            }
-          }
+        for (int q2 = 0; q2 < 8; ++q2)
+          if (q2 < S) ld_cluster_f32x4x2(tok_base, ca * 4, cb * 4, q2, v[q2]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) z[k] = v[0][k];
+#pragma unroll
+        for (int q2 = 1; q2 < 8; ++q2)
+          if (q2 < S)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) z[k] += v[q2][k];
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = (k < 4 ? ca : cb) + (k & 3);
+        if (c < N_r) {
+          const float sg = sigmoid_fast(z[k]);
+          if (k < 4) topk_insert_ki(ka, ia, sg + sm.bias[c], c);
+          else topk_insert_ki(kb2, ib, sg + sm.bias[c], c);
+          if (srow != nullptr) srow[c] = sg;
         }
       }
+    }
 #pragma unroll
-      for (int c = 1; c < SUB; ++c)
+    for (int j = 0; j < KMAX; ++j)
+      if (ib[j] < N_r) topk_insert_lex(ka, ia, kb2[j], ib[j]);
+    for (int m = 1; m < TPT; m <<= 1) {
+      float pk[KMAX];
+      int pi[KMAX];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (ii[c][j] < N_r) topk_insert_ki(kk[0], ii[0], kk[c][j], ii[c][j]);
-      float (&kk0)[KMAX] = kk[0];
-      int (&ii0)[KMAX] = ii[0];
-      // the upper half hands its list to the lower half, which merges: every
-      // upper-half index exceeds every lower-half one, and the list arrives
-      // in (key desc, index asc) order, so equal keys stay lowest-index first
-      if (half == 1) {
+      for (int j = 0; j < KMAX; ++j) {
+        pk[j] = __shfl_xor_sync(0xffffffffu, ka[j], m);
+        pi[j] = __shfl_xor_sync(0xffffffffu, ia[j], m);
+      }
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-          sm.m_key[j][r] = kk0[j];
-          sm.m_idx[j][r] = ii0[j];
+      for (int j = 0; j < KMAX; ++j)
+        if (pi[j] < N_r) topk_insert_lex(ka, ia, pk[j], pi[j]);
+    }
+    if (ch == 0 && tt < T) {
+      // the affinities of the selected experts, from the same summed logits
+      float ss[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        float zz = 0.0f;
+        if (ia[j] < N_r) {
+          const uint32_t o = static_cast<uint32_t>(ia[j]) * 4;
+          if (S == 1) zz = park[rr * PR + ia[j]];
+          else
+            for (int q2 = 0; q2 < S; ++q2) zz += ld_cluster_f32(tok_base + o, q2);
         }
+        ss[j] = ia[j] < N_r ? sigmoid_fast(zz) : 0.0f;
       }
-      mbar_arrive(&sm.xbar);
-      if (half == 0 && warp_wait(&sm.xbar, 0, abort)) {
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (sm.m_idx[j][r] < N_r) topk_insert_ki(kk0, ii0, sm.m_key[j][r], sm.m_idx[j][r]);
-        // the affinities of the selected experts, recomputed from the parked
-        // logits ([expert][token], both halves) exactly as for their keys
-        const float* logits = reinterpret_cast<const float*>(tiles);
-        float ss0[KMAX];
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) ss0[j] = ii0[j] < N_r ? sigmoid_fast(logits[ii0[j] * BM + r]) : 0.0f;
-        if (t < T) topk_store(ii0, ss0, K, topk_idx + static_cast<size_t>(t) * K, gates + static_cast<size_t>(t) * K);
-      }
+      topk_store(ia, ss, K, topk_idx + static_cast<size_t>(tt) * K, gates + static_cast<size_t>(tt) * K);
     }
   }
   if (S > 1) {
