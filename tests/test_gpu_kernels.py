@@ -116,13 +116,18 @@ def _check_routing(gpu_idx, s64, b, K, margin=1e-5):
     return diff
 
 
-@pytest.mark.parametrize("name,T", [("tiny", None), ("mid", None), ("mid", 1000), ("mid", 5000), ("prefill", 1500),
-                                    ("decode", None)])
-def test_router_tensor_cores(lib, name, T):
+@pytest.mark.parametrize("name,T,K", [("tiny", None, None), ("mid", None, None), ("mid", 1000, None),
+                                      ("mid", 5000, None), ("prefill", 1500, None), ("decode", None, None),
+                                      # top-K lists of 16 (K_r > 8): one tile (cluster of 8), and 40 tiles
+                                      ("mid", 128, 12), ("mid", 5000, 16)])
+def test_router_tensor_cores(lib, name, T, K):
+    import dataclasses
     from fine_grained_fp8_sigmoid_b200 import binding as B
     cfg = workloads.CONFIGS[name]
     if T is not None:
         cfg = cfg.with_tokens(T)
+    if K is not None:
+        cfg = dataclasses.replace(cfg, K_r=K)
     u, e, b = workloads.activations(cfg), workloads.centroids(cfg), workloads.bias(cfg)
     idx = torch.empty(cfg.T, cfg.K_r, dtype=torch.int32, device="cuda")
     gates = torch.empty(cfg.T, cfg.K_r, dtype=torch.float32, device="cuda")
