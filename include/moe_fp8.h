@@ -118,8 +118,13 @@ MOE_API int moe_quant_128x128(const float* w, int rows, int cols, uint8_t* q,
  *              descending, equal keys by lower index first
  *   gates      [T][K_r] FP32: g = s_sel / sum(s_sel), in the same order
  * The logits u . e run on the tensor cores in BF16 with FP32 accumulation; the
- * key s + b is formed in FP32. Limits: 1 <= K_r <= 16, K_r <= N_r <= 256,
- * d a multiple of 64.
+ * affinity uses the hardware exponential and reciprocal (relative error
+ * ~1e-6); the key s + b is formed in FP32. With few 128-token tiles the launch
+ * is a set of thread-block clusters (2..8 CTAs per tile) that split d and add
+ * their partial logits in a fixed order, so results do not depend on the
+ * schedule. Limits: 1 <= K_r <= 16, K_r <= N_r <= 256, d a multiple of 64.
+ * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED before any launch;
+ * MOE_ERR_CUDA if the launch fails (moe_last_error_detail names the call).
  */
 MOE_API int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
               const float* scores_in, int T, int d, int N_r, int K_r,
