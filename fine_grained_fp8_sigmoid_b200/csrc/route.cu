@@ -28,6 +28,8 @@
 // rank's shared memory alive until all ranks have read it.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
 // epilogue (TMEM lane quadrant w%4, column half (w-4)/4 while reading TMEM).
+#include <mutex>
+
 #include "host.cuh"
 
 namespace moe {
@@ -481,9 +483,14 @@ extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
   if (int st = cuda_status(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                            "router smem attribute"))
     return st;
-  // split K over a cluster of S CTAs per token tile while the SMs allow
-  int S = 1;
-  while (S < 8 && tiles * S * 2 <= di.sm_count && S * 2 <= NG_all) S *= 2;
+  // split K over a cluster of S CTAs per token tile while the SMs allow, up
+  // to the largest cluster the device can place (queried once per device and
+  // kernel variant)
+  static std::mutex mu;
+  static int max_cluster[64][2] = {};
+  int dev = 0;
+  if (int st = cuda_status(cudaGetDevice(&dev), "cudaGetDevice")) return st;
+  if (dev < 0 || dev >= 64) return MOE_ERR_NO_DEVICE;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.blockDim = dim3(THREADS);
@@ -492,15 +499,27 @@ extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  for (;; S /= 2) {   // a cluster size the device can place
-    cfg.gridDim = dim3(tiles * S);
-    attr[0].val.clusterDim.x = S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    int n_clusters = 0;
-    if (S == 1 || (cudaOccupancyMaxActiveClusters(&n_clusters, k, &cfg) == cudaSuccess && n_clusters > 0)) break;
-    cudaGetLastError();
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  const int variant = K_r <= 8 ? 0 : 1;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (max_cluster[dev][variant] == 0) {
+      int m = 8;
+      for (; m > 1; m /= 2) {
+        cfg.gridDim = dim3(m);
+        attr[0].val.clusterDim.x = m;
+        int n_clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&n_clusters, k, &cfg) == cudaSuccess && n_clusters > 0) break;
+        cudaGetLastError();
+      }
+      max_cluster[dev][variant] = m;
+    }
   }
+  int S = 1;
+  while (S < max_cluster[dev][variant] && tiles * S * 2 <= di.sm_count && S * 2 <= NG_all) S *= 2;
+  cfg.gridDim = dim3(tiles * S);
+  attr[0].val.clusterDim.x = S;
   if (int st = cuda_status(cudaLaunchKernelEx(&cfg, k, tm_u, tm_e, b, T, d, N_r, K_r, S, scores_out, topk_idx, gates),
                            "router launch"))
     return st;
