@@ -97,3 +97,51 @@ class MoELayerFP8:
         self.forward(u_dev, e, b, update_bias, stream)
         out_host.copy_(self.out, non_blocking=True)
         return out_host
+
+    def forward_host_pipelined(self, u_hosts, e, b, out_hosts, u_devs, update_bias=True):
+        """End to end over a sequence of batches in pinned host memory, with the
+        copies overlapped with the kernels: batch i+1's input goes to the
+        device, and batch i-1's h' to the host, on a copy stream while batch i
+        runs on the current stream. u_devs holds two device input buffers. On
+        return everything is enqueued; out_hosts[i] holds batch i's h' once the
+        current stream is synchronised."""
+        comp = torch.cuda.current_stream(self.device)
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream(self.device)
+        copy = self._copy_stream
+        n = len(u_hosts)
+        h2d_done = [torch.cuda.Event(), torch.cuda.Event()]   # input buffer k filled
+        read_done = [torch.cuda.Event(), torch.cuda.Event()]  # input buffer k no longer read
+        out_ready, d2h_done = torch.cuda.Event(), torch.cuda.Event()
+        copy.wait_stream(comp)            # inputs and buffers as the caller left them
+        with torch.cuda.stream(copy):
+            u_devs[0].copy_(u_hosts[0], non_blocking=True)
+            h2d_done[0].record(copy)
+        for i in range(n):
+            k = i % 2
+            if i + 1 < n:
+                with torch.cuda.stream(copy):
+                    if i >= 1:            # batch i-1 used the buffer batch i+1 fills
+                        copy.wait_event(read_done[(i + 1) % 2])
+                    u_devs[(i + 1) % 2].copy_(u_hosts[i + 1], non_blocking=True)
+                    h2d_done[(i + 1) % 2].record(copy)
+            comp.wait_event(h2d_done[k])
+            self.route(u_devs[k], e, b)
+            self.quant(u_devs[k])
+            self.permute()
+            self.experts()
+            if i >= 1:                    # batch i-1's h' has left self.out
+                comp.wait_event(d2h_done)
+            self.combine(u_devs[k])
+            read_done[k].record(comp)
+            out_ready.record(comp)
+            if update_bias:
+                self.bias_update(b)
+            with torch.cuda.stream(copy):
+                copy.wait_event(out_ready)
+                out_hosts[i].copy_(self.out, non_blocking=True)
+                d2h_done.record(copy)
+        comp.wait_event(d2h_done)
+        for t in u_devs:
+            t.record_stream(copy)
+        return out_hosts
