@@ -110,3 +110,27 @@ def test_layer_mid_sampled(lib):
 def test_layer_full_size_sampled(lib, name, n):
     cfg = workloads.CONFIGS[name]
     _run(cfg, _sample(cfg, n, seed=3), weights_on="cuda")
+
+
+def test_layer_pipelined_host_path_matches_plain():
+    """forward_host_pipelined (copies on a second stream, two input buffers)
+    gives, batch for batch and bit for bit, what forward_host gives, bias
+    updates included."""
+    cfg = workloads.CONFIGS["tiny"]
+    layer = _build(cfg, "cuda")
+    u = workloads.activations(cfg, device="cuda")
+    e = workloads.centroids(cfg, device="cuda")
+    b = workloads.bias(cfg, device="cuda")
+    u_hosts = [u.cpu().pin_memory(), torch.roll(u, 1, 0).cpu().pin_memory(), (u * 0.5).cpu().pin_memory()]
+    outs = [torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in u_hosts]
+    refs = [torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in u_hosts]
+    b_pipe, b_plain = b.clone(), b.clone()
+    layer.forward_host_pipelined(u_hosts, e, b_pipe, outs, [torch.empty_like(u), torch.empty_like(u)])
+    torch.cuda.synchronize()
+    u_dev = torch.empty_like(u)
+    for src, ref in zip(u_hosts, refs):
+        layer.forward_host(src, e, b_plain, ref, u_dev)
+    torch.cuda.synchronize()
+    for i, (o, r) in enumerate(zip(outs, refs)):
+        assert torch.equal(o, r), f"batch {i}"
+    assert torch.equal(b_pipe, b_plain)
