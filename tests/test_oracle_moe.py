@@ -263,6 +263,30 @@ def test_expert_ffn_closed_form():
     assert np.all(y == 448.0 * scale)
 
 
+def test_expert_ffn_gate_and_up_roles():
+    # SwiGLU is silu(G) * U with G from W_gate and U from W_up, not the other
+    # way round. d = 256, I = 128; row 0 is x = 1, row 1 is x = 1/2 (code 0x38
+    # with scales 1 and 0.5). W_gate = 2^-7 (code 0x04) and W_up = 2^-8 (code
+    # 0x02) everywhere, so row 0 has G = 2, U = 1 and row 1 has G = 1, U = 1/2.
+    # A negative up weight (code 0x82) flips U. Each intermediate tile holds
+    # one value a, requantised to +-448 with scale fl32(|a|/448); W_down =
+    # 2^-7 (code 0x04) sums I = 128 of them: y = +-448 * scale (exact).
+    d, I = 256, 128
+    xq = np.full((2, d), 0x38, np.uint8)
+    xs = np.array([[1.0, 1.0], [0.5, 0.5]])
+    sig = lambda v: 1.0 / (1.0 + math.exp(-v))
+    for up_code, sign in [(0x02, 1.0), (0x82, -1.0)]:
+        y, h = moe.expert_ffn(xq, xs, _const_expert(d, I, 0x04, up_code, 0x04))
+        for row, (G, U) in enumerate([(2.0, 1.0), (1.0, 0.5)]):
+            a = float(np.float32(G * sig(G) * U * sign))
+            swapped = float(np.float32(U * sig(U) * G * sign))
+            assert a != swapped
+            scale = float(np.float32(abs(a) / 448.0))
+            assert np.all(h[row] == math.copysign(448.0 * scale, a)), row
+            assert np.all(y[row] == math.copysign(448.0 * scale, a)), row
+            assert y.shape == (2, d) and h.shape == (2, I)
+
+
 def test_expert_ffn_zero_gate_gives_zero():
     xq = encode(np.random.default_rng(0).standard_normal((4, 256)))
     y, h = moe.expert_ffn(xq, np.ones((4, 2)), _const_expert(256, 128, 0x00, 0x38, 0x38))
