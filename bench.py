@@ -121,25 +121,33 @@ def workload_desc(cfg):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 20 ms)
+    around a region; summary() keeps the samples taken between mark_start()
+    and mark_end() (nvidia-smi stamps each sample with the wall clock)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_ms: int = 20):
         self.index = index
+        self.period_ms = period_ms
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.time() + 10.0        # nvidia-smi takes a moment to start
+            while not self.lines and time.time() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
@@ -148,33 +156,50 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(2.5 * self.period_ms / 1e3)   # the samples of the region's last moments
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    @staticmethod
+    def parse(lines, t0=None, t1=None):
+        """Median SM clock, max clock and throttle reasons of the samples whose
+        timestamp lies in [t0, t1] (epoch seconds; None: no bound)."""
+        import datetime
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                clk, cmax = float(parts[2]), float(parts[3])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            if (t0 is not None and ts < t0 - 0.02) or (t1 is not None and ts > t1 + 0.02):
+                continue
+            sm.append(clk)
+            mx = cmax
+            for n, v in zip(ClockSampler.REASONS, parts[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+    def summary(self):
+        return self.parse(self.lines, self.t0, self.t1)
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -229,20 +254,50 @@ def time_oracle(cfg, n_tokens, steps, device="cuda"):
 
 # ---------------------------------------------------------------- GPU arm
 
-def run_ours(args, rank, world, local_rank):
-    import numpy as np
-    import torch
-    import torch.distributed as dist
+NOMINAL_FP8_TFLOPS = 4500.0     # dense FP8 on B200 (NVIDIA's figure without sparsity)
+NOMINAL_HBM_GBS = 8000.0
 
+
+def roofline(cfg, gemm_s, touched, peaks):
+    """Roofline of the grouped GEMM (one moe_grouped_gemm_fp8 call, 2 launches)
+    from its average device time. The roof is the slower of the two ideal
+    times: algorithmic FLOPs at the dense FP8 peak, and algorithmic bytes at
+    the measured copy bandwidth; "bound" names it, and "frac" is the achieved
+    rate over it. The FP8 peak is the measured burst figure (dense FP8 = 2 x
+    the measured BF16 GEMM rate, the nominal ratio): the timed regions are
+    well under a second of back-to-back steps, not the seconds-long
+    power-capped loop of the sustained figure. Fractions of the FP8 peak
+    (burst, sustained, nominal) and of the HBM bandwidth are reported beside
+    it whichever bound applies."""
+    flops = layer_flops(cfg)
+    nbytes = gemm_algorithmic_bytes(cfg, touched)
+    fp8_burst = 2.0 * peaks["bf16"]
+    fp8_sust = 2.0 * peaks["bf16_sustained"]
+    tf = flops / gemm_s / 1e12
+    gbs = nbytes / gemm_s / 1e9
+    t_tensor = flops / (fp8_burst * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    common = {"gemm_ms": gemm_s * 1e3, "gemm_tflops": tf, "gemm_gbs": gbs,
+              "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+              "ideal_ms_tensor": t_tensor * 1e3, "ideal_ms_hbm": t_hbm * 1e3,
+              "frac_of_fp8_burst": tf / fp8_burst, "frac_of_fp8_sustained": tf / fp8_sust,
+              "frac_of_fp8_nominal": tf / NOMINAL_FP8_TFLOPS,
+              "frac_of_hbm": gbs / peaks["hbm_gbs"], "frac_of_hbm_nominal": gbs / NOMINAL_HBM_GBS,
+              "experts_touched": touched + 1}
+    if t_tensor >= t_hbm:
+        return dict({"bound": "tensor", "achieved": tf, "peak": fp8_burst, "unit": "TFLOP/s",
+                     "frac": tf / fp8_burst,
+                     "peak_source": f"bf16 burst {peaks['bf16']} TF/s x2 (of {peaks['source']})"},
+                    **common)
+    return dict({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                 "frac": gbs / peaks["hbm_gbs"],
+                 "peak_source": f"copy bandwidth {peaks['hbm_gbs']} GB/s (of {peaks['source']})"},
+                **common)
+
+
+def build_layer(cfg, dev):
     import workloads
     from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
-    from fine_grained_fp8_sigmoid_b200 import binding as B
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    cfg = workloads.CONFIGS[args.workload]
-    peaks = _peaks()
-
     layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, device=dev)
     for slot in range(cfg.N_r + 1):
         w = workloads.expert_weights(cfg, slot, device=dev)
@@ -251,30 +306,34 @@ def run_ours(args, rank, world, local_rank):
     u = workloads.activations(cfg, device=dev)
     e = workloads.centroids(cfg, device=dev)
     b0 = workloads.bias(cfg, device=dev)
-    b = b0.clone()
+    return layer, u, e, b0
+
+
+def time_layer(layer, u, e, b, steps, warmup, dev, world, local_rank):
+    """Times `steps` layer steps (after `warmup`), CUDA events on the launching
+    stream, a barrier and a synchronize on both sides. Returns (ms per step,
+    max over ranks; mean GEMM ms; clock summary)."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from fine_grained_fp8_sigmoid_b200 import binding as B
     stream = torch.cuda.current_stream(dev)
-    torch.cuda.synchronize(dev)
-
-    def step():
+    for _ in range(warmup):
         layer.forward(u, e, b, update_bias=True)
-
-    for _ in range(args.warmup):
-        step()
     torch.cuda.synchronize(dev)
-    gemm_launches = B.moe_grouped_gemm_fp8_launches(cfg.d, cfg.I)
     if B.moe_get_error() != 0:
         raise RuntimeError("device error word set during warm-up")
-
-    K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+          for _ in range(steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        clk.mark_start()
         start.record(stream)
-        for i in range(K):
+        for i in range(steps):
             layer.route(u, e, b)
             layer.quant(u)
             layer.permute()
@@ -285,64 +344,45 @@ def run_ours(args, rank, world, local_rank):
             layer.bias_update(b)
         stop.record(stream)
         torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+        clk.mark_end()
+        if world > 1:
+            dist.barrier()
     ms_total = max_over_ranks(start.elapsed_time(stop), dev)
-    gemm_ms = [a.elapsed_time(z) for a, z in ev]
+    gemm_ms = float(np.mean([a.elapsed_time(z) for a, z in ev]))
     if B.moe_get_error() != 0:
         raise RuntimeError("device error word set during the timed region")
-    ms_step = ms_total / K
-    tokens_per_s = whole_job_tokens_per_s(cfg.T, world, ms_step)
+    return ms_total / steps, gemm_ms, clk.summary()
 
-    flops = layer_flops(cfg)
-    gemm_avg_s = float(np.mean(gemm_ms)) / 1e3
-    # dense FP8 = 2x dense BF16 (nominal ratio). The GEMM is timed inside a
-    # long run of back-to-back steps under the power cap, so the sustained
-    # figure is its denominator; the burst one is reported beside it.
-    fp8_peak = 2.0 * peaks["bf16_sustained"]
-    fp8_burst = 2.0 * peaks["bf16"]
-    achieved_tf = flops / gemm_avg_s / 1e12
-    layer_tf = flops / (ms_step / 1e3) / 1e12
-    touched = int((layer.counts > 0).sum().item())
-    gemm_bytes = gemm_algorithmic_bytes(cfg, touched)
-    achieved_gbs = gemm_bytes / gemm_avg_s / 1e9
-    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)      # FLOP per byte
-    if flops / gemm_bytes >= ridge:
-        roof = {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak, "unit": "TFLOP/s",
-                "frac": achieved_tf / fp8_peak,
-                "peak_source": f"{peaks['source']} bf16 sustained {peaks['bf16_sustained']} TF/s x2",
-                "frac_of_burst": achieved_tf / fp8_burst}
-    else:
-        roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved_gbs / peaks["hbm_gbs"],
-                "peak_source": f"{peaks['source']} copy bandwidth {peaks['hbm_gbs']} GB/s"}
 
-    balance = None
-    if cfg.name == "skew":
-        # the auxiliary-loss-free balancing run: 100 steps of route -> experts ->
-        # bias update from the initial bias, max/mean expert load of each step
-        b.copy_(b0)
-        ratios = torch.zeros(100, device=dev)
-        for i in range(100):
-            layer.forward(u, e, b, update_bias=True)
-            ratios[i].copy_(layer.max_over_mean[0])
-        r = ratios.cpu().tolist()
-        balance = {"steps": 100, "gamma": 0.001, "max_over_mean_first": r[0],
-                   "max_over_mean_last": r[-1], "max_over_mean_min": min(r),
-                   "max_over_mean_every_10": r[::10]}
+def balance_run(layer, u, e, b, b0, steps=100):
+    """The auxiliary-loss-free balancing run: `steps` steps of route ->
+    experts -> bias update from the initial bias; max/mean expert load of
+    every step (read back once at the end)."""
+    import torch
+    b.copy_(b0)
+    ratios = torch.zeros(steps, device=u.device)
+    for i in range(steps):
+        layer.forward(u, e, b, update_bias=True)
+        ratios[i].copy_(layer.max_over_mean[0])
+    r = ratios.cpu().tolist()
+    return {"steps": steps, "gamma": 0.001, "max_over_mean_first": r[0],
+            "max_over_mean_last": r[-1], "max_over_mean_min": min(r),
+            "max_over_mean_every_10": r[::10], "max_over_mean_per_step": r}
 
-    # end to end through the public API: every step copies its u from pinned
-    # host memory in and its h' out. The pipelined form overlaps those copies
-    # with the kernels (a copy stream, two device input buffers); it is first
-    # checked bit for bit against the plain form, which is the fallback.
+
+def e2e_run(layer, u, e, b, b0, steps, dev, world, cfg):
+    """End to end through the public API: every step copies its u from pinned
+    host memory in and its h' out. The pipelined form overlaps those copies
+    with the kernels (a copy stream, two device input buffers); it is first
+    checked bit for bit against the plain form, which is the fallback."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
     u_host = u.cpu().pin_memory()
     out_host = torch.empty(cfg.T, cfg.d, dtype=torch.bfloat16).pin_memory()
     u_dev = torch.empty_like(u)
-    Ke = max(3, K // 2)
-    e2e_mode = "copies overlapped with the kernels (copy stream, double-buffered input)"
+    mode = "copies overlapped with the kernels (copy stream, double-buffered input)"
     try:
         u_devs = [torch.empty_like(u), torch.empty_like(u)]
-        # check: two different batches, no bias update, against the plain path
         u_host2 = torch.roll(u, shifts=1, dims=0).cpu().pin_memory()
         outs = [torch.empty_like(out_host).pin_memory() for _ in range(2)]
         refs = [torch.empty_like(out_host).pin_memory() for _ in range(2)]
@@ -359,31 +399,110 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        layer.forward_host_pipelined([u_host] * Ke, e, b, [out_host] * Ke, u_devs)
+        layer.forward_host_pipelined([u_host] * steps, e, b, [out_host] * steps, u_devs)
         e1.record(stream)
         torch.cuda.synchronize(dev)
     except Exception as exc:   # the plain, serialised form
-        e2e_mode = f"serialised copies (pipelined form unavailable: {exc})"
+        mode = f"serialised copies (pipelined form unavailable: {exc})"
         b.copy_(b0)
         for _ in range(2):
             layer.forward_host(u_host, e, b, out_host, u_dev)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(Ke):
+        for _ in range(steps):
             layer.forward_host(u_host, e, b, out_host, u_dev)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, dev)
-    e2e_tps = whole_job_tokens_per_s(cfg.T, world, e2e_ms)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
+    return {"value": whole_job_tokens_per_s(cfg.T, world, ms), "unit": "tokens/s",
+            "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2,
+            "steps": steps, "mode": mode}
+
+
+def sub_workload(name, args, dev, world, local_rank, peaks):
+    """One more workload of the same layer shape, measured in the same run:
+    decode (the HBM-bound weight stream) or skew (with its balancing run)."""
+    import torch
+
+    import workloads
+    cfg = workloads.CONFIGS[name]
+    layer, u, e, b0 = build_layer(cfg, dev)
+    b = b0.clone()
+    ms_step, gemm_ms, clocks = time_layer(layer, u, e, b, args.steps, args.warmup, dev, world,
+                                          local_rank)
+    touched = int((layer.counts > 0).sum().item())
+    roof = roofline(cfg, gemm_ms / 1e3, touched, peaks)
+    res = {"workload": workload_desc(cfg), "T": cfg.T, "steps": args.steps,
+           "value": whole_job_tokens_per_s(cfg.T, world, ms_step), "unit": "tokens/s",
+           "ms_per_step": ms_step, "tflops": layer_flops(cfg) / (ms_step / 1e3) / 1e12,
+           "roofline": roof, "clocks": clocks}
+    if name == "decode":
+        res["gemm_weight_stream"] = {"gb_per_call": roof["algorithmic_bytes"] / 1e9,
+                                     "gbs": roof["gemm_gbs"],
+                                     "frac_of_measured_hbm": roof["gemm_gbs"] / peaks["hbm_gbs"],
+                                     "frac_of_8tbs": roof["gemm_gbs"] / NOMINAL_HBM_GBS}
+    if name == "skew":
+        res["balance"] = balance_run(layer, u, e, b, b0)
+    del layer, u, e, b, b0
+    torch.cuda.empty_cache()
+    return res
+
+
+def workload_config(args):
+    """The named workload, with the profiling overrides of --experts/--tokens
+    (a smaller layer whose kernels see the same shapes per token)."""
+    import dataclasses
+
+    import workloads
+    cfg = workloads.CONFIGS[args.workload]
+    if args.experts is not None:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_e{args.experts}", N_r=args.experts)
+    if args.tokens is not None:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}_t{args.tokens}", T=args.tokens)
+    return cfg
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    import workloads
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workload_config(args)
+    peaks = _peaks()
+
+    layer, u, e, b0 = build_layer(cfg, dev)
+    b = b0.clone()
+    torch.cuda.synchronize(dev)
+    gemm_launches = B.moe_grouped_gemm_fp8_launches(cfg.d, cfg.I)
+    K = args.steps
+    ms_step, gemm_ms, clocks = time_layer(layer, u, e, b, K, args.warmup, dev, world, local_rank)
+    tokens_per_s = whole_job_tokens_per_s(cfg.T, world, ms_step)
+    touched = int((layer.counts > 0).sum().item())
+    roof = roofline(cfg, gemm_ms / 1e3, touched, peaks)
+    layer_tf = layer_flops(cfg) / (ms_step / 1e3) / 1e12
+    balance = balance_run(layer, u, e, b, b0) if cfg.name == "skew" else None
+    e2e = e2e_run(layer, u, e, b, b0, max(3, K // 2), dev, world, cfg)
+    del layer, u, e, b, b0
+    torch.cuda.empty_cache()
+
+    # the decode and skew workloads of the same layer shape, as sub-results
+    extra = {}
+    if cfg == workloads.CONFIGS[CONFIG_NAME] and not args.no_sub_workloads:
+        for name in ("decode", "skew"):
+            extra[name] = sub_workload(name, args, dev, world, local_rank, peaks)
 
     result = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             tps, dt, desc = time_oracle(cfg, n_tokens=1, steps=3, device=dev)
-            cpu = {"value": tps, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
-                   "sample": desc, "seconds_per_step": dt}
+            cpu = {"value": tps, "unit": "tokens/s", "cores": os.cpu_count(),
+                   "blas_threads": _blas_threads(), "kind": "oracle", "sample": desc,
+                   "seconds_per_step": dt}
         result = {
             "metric": METRIC,
             "value": tokens_per_s,
@@ -403,21 +522,18 @@ def run_ours(args, rank, world, local_rank):
                        "l2": f"inputs larger than L2: {weight_bytes(cfg) / 1e9:.2f} GB of expert "
                              "weights stream every step"},
             "tflops": layer_tf,
-            "pct_fp8_peak": layer_tf / fp8_peak,
+            "pct_fp8_peak": layer_tf / (2.0 * peaks["bf16"]),
             "roofline": dict(roof, kernel=f"moe_grouped_gemm_fp8 ({gemm_launches} launches)",
-                             traffic=gemm_traffic(cfg), gemm_ms=float(np.mean(gemm_ms)),
-                             gemm_tflops=achieved_tf, algorithmic_bytes=gemm_bytes,
-                             experts_touched=touched + 1),
+                             traffic=gemm_traffic(cfg)),
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_tps, "unit": "tokens/s",
-                    "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2,
-                    "steps": Ke, "mode": e2e_mode},
+            "e2e": e2e,
             # quant, router, permute (count, scan, scatter, gather), the GEMM's
             # launches, combine, bias update
             "gpu_launches": (8 + gemm_launches) * K,
             "balance": balance,
-            "clocks": clk.summary(),
+            "clocks": clocks,
         }
+        result.update(extra)
     return result
 
 
@@ -455,27 +571,55 @@ def run_reference(args, rank, world):
         "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "T": cfg.T, "d": cfg.d, "N_r": cfg.N_r,
                    "K_r": cfg.K_r, "I": cfg.I, "N_s": 1, "sample_tokens": n_tokens},
-        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": _blas_threads(),
-                         "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": os.cpu_count(),
+                         "blas_threads": _blas_threads(), "kind": "oracle", "sample": desc},
         "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
-def main():
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(nproc: int, script: str, argv) -> int:
+    """Runs `script argv` as nproc ranks on this node under torch.distributed.run
+    (rendezvous on 127.0.0.1), bounded by a timeout; returns its exit status."""
+    cmd = ["timeout", "-k", "60", "1800", sys.executable, "-m", "torch.distributed.run",
+           "--nnodes=1", f"--nproc-per-node={nproc}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), script, *argv]
+    return subprocess.call(cmd)
+
+
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-workloads", action="store_true",
+                    help="measure only the main workload (not decode and skew beside prefill)")
     ap.add_argument("--workload", default=CONFIG_NAME,
                     help="prefill (the benchmark) or a smaller layer for profiling: mid, decode, tiny")
-    args = ap.parse_args()
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling only: the workload with this many routed experts")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="profiling only: the workload with this many tokens")
+    argv = sys.argv[1:] if argv is None else argv
+    args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: re-run this script as args.gpus ranks
+        sys.exit(launch_ranks(args.gpus, os.path.abspath(sys.argv[0]), argv))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
 
     if args.impl == "reference":
         res = run_reference(args, rank, world)
@@ -488,9 +632,12 @@ def main():
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local_rank))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        else:   # the rank plumbing on CPU (tests)
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=300))
     try:
         res = run_ours(args, rank, world, local_rank)
     finally:

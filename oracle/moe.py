@@ -234,7 +234,7 @@ def bias_update(b, counts, T: int, K: int, gamma: float = GAMMA):
 # Whole layer
 # --------------------------------------------------------------------------
 
-def moe_forward(u, e, b, K: int, weights, tokens=None, select=None) -> dict:
+def moe_forward(u, e, b, K: int, weights, tokens=None, select=None, map_fn=map) -> dict:
     """The layer's forward pass.
 
     u [T, d], e [N_r, d] (bf16 values), b [N_r] (FP32 values).
@@ -246,6 +246,9 @@ def moe_forward(u, e, b, K: int, weights, tokens=None, select=None) -> dict:
     top-K (to evaluate a token under another, equally valid, selection when
     two keys are closer than the comparison can resolve); gates are still the
     oracle's affinities normalised over that selection.
+    map_fn: how the per-expert FFNs are evaluated (the builtin map, or an
+    executor's map to run independent experts side by side; the arithmetic
+    of each expert is the same either way).
     """
     u = np.asarray(u, np.float64)
     T, d = u.shape
@@ -260,20 +263,25 @@ def moe_forward(u, e, b, K: int, weights, tokens=None, select=None) -> dict:
     sample = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
     S = sample.shape[0]
     xq, xs = quant_1x128(u[sample])
-    I = None
     y_routed = np.zeros((S, K, d))
     h_routed = None
     sel = idx[sample]
-    for slot in np.unique(sel):
-        who = np.argwhere(sel == slot)           # rows (sample i, k)
-        w = weights(int(slot))
-        I = w["gate_q"].shape[0]
-        y, h = expert_ffn(xq[who[:, 0]], xs[who[:, 0]], w)
+    slots = [int(s_) for s_ in np.unique(sel)]
+    whos = [np.argwhere(sel == slot) for slot in slots]      # rows (sample i, k)
+
+    def one(j):
+        if j == len(slots):
+            return expert_ffn(xq, xs, weights(N_r))
+        who = whos[j]
+        return expert_ffn(xq[who[:, 0]], xs[who[:, 0]], weights(slots[j]))
+
+    results = list(map_fn(one, range(len(slots) + 1)))
+    for who, (y, h) in zip(whos, results[:-1]):
         if h_routed is None:
-            h_routed = np.zeros((S, K, I))
+            h_routed = np.zeros((S, K, h.shape[1]))
         y_routed[who[:, 0], who[:, 1]] = y
         h_routed[who[:, 0], who[:, 1]] = h
-    y_shared, h_shared = expert_ffn(xq, xs, weights(N_r))
+    y_shared, h_shared = results[-1]
 
     acc = u[sample] + y_shared
     for k in range(K):

@@ -24,9 +24,36 @@ def test_gemm_algorithmic_bytes_terms():
     assert abs(bench.gemm_algorithmic_bytes(cfg, 256) / 1e9 - 14.29) < 0.01
 
 
-def test_prefill_is_tensor_bound_and_decode_hbm_bound():
-    peaks = bench._peaks()
-    ridge = 2 * peaks["bf16_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+def test_roofline_bound_is_the_slower_ideal_time():
+    peaks = dict(hbm_gbs=6540.0, bf16=1631.7, bf16_sustained=1358.8, source="measured")
     pre, dec = workloads.CONFIGS["prefill"], workloads.CONFIGS["decode"]
-    assert bench.layer_flops(pre) / bench.gemm_algorithmic_bytes(pre, 256) > ridge
-    assert bench.layer_flops(dec) / bench.gemm_algorithmic_bytes(dec, 256) < ridge
+    # prefill: 6.494 TFLOP at 3263.4 TF/s = 1.99 ms; 14.29 GB at 6540 GB/s = 2.19 ms
+    r = bench.roofline(pre, 5.917e-3, 256, peaks)
+    assert abs(r["ideal_ms_tensor"] - 1.990) < 1e-3 and abs(r["ideal_ms_hbm"] - 2.185) < 1e-3
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6540.0
+    assert r["frac"] == r["achieved"] / 6540.0 == r["frac_of_hbm"]
+    assert r["gemm_tflops"] == bench.layer_flops(pre) / 5.917e-3 / 1e12
+    assert abs(r["frac_of_fp8_burst"] - 0.3363) < 1e-3           # 1097.5 / 3263.4
+    assert abs(r["frac_of_fp8_sustained"] - 0.4038) < 1e-3
+    assert abs(r["frac_of_fp8_nominal"] - 1097.5 / 4500) < 1e-3
+    # with a faster copy the same call is tensor-bound, against the burst peak
+    t = bench.roofline(pre, 5.917e-3, 256, dict(peaks, hbm_gbs=8000.0))
+    assert t["bound"] == "tensor" and t["peak"] == 2 * 1631.7 and t["frac"] == t["frac_of_fp8_burst"]
+    d = bench.roofline(dec, 1.9e-3, 256, peaks)
+    assert d["bound"] == "hbm" and d["ideal_ms_hbm"] > 10 * d["ideal_ms_tensor"]
+
+
+def test_clock_samples_inside_the_region_only():
+    import datetime
+    t0 = datetime.datetime(2026, 1, 2, 3, 4, 5).timestamp()
+
+    def line(dt, mhz, cap="Not Active"):
+        ts = datetime.datetime.fromtimestamp(t0 + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {mhz}, 1965, 900.0, 0x0, Not Active, Not Active, Not Active, {cap}"
+
+    lines = [line(-1.0, 300), line(0.05, 1900), line(0.1, 1500, "Active"), line(0.15, 1700),
+             line(2.0, 300)]
+    s = bench.ClockSampler.parse(lines, t0, t0 + 0.2)
+    assert s["samples"] == 3 and s["sm_mhz"] == 1700 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    assert bench.ClockSampler.parse([], t0, t0 + 1)["reasons"] == ["unsampled"]

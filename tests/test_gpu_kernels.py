@@ -143,6 +143,73 @@ def test_router_tensor_cores(lib, name, T, K):
     assert np.allclose(gates.cpu().double().numpy(), rg, rtol=1e-4, atol=1e-6)
 
 
+def _tied_centroids(cfg, mode):
+    """Centroids with exactly repeated rows, so that logits (and with equal
+    bias, keys) tie bit for bit. mode "pairs": a few expert pairs share a
+    row, chosen to fall in different threads, warps and column halves of
+    the fused router; mode "groups": only 4 distinct rows, each repeated
+    N_r/4 times, so every selection breaks ties."""
+    e = workloads.centroids(cfg).clone()
+    b = workloads.bias(cfg).clone()
+    N = cfg.N_r
+    if mode == "pairs":
+        pairs = [(0, N - 1), (2, 3), (5, N // 2), (7, N // 2 + 7), (N // 4, N // 4 + 4), (1, N - 2)]
+        for lo, hi in pairs:
+            e[hi] = e[lo]
+            b[hi] = b[lo]
+        return e, b, pairs
+    e = e[torch.arange(N) % 4].clone()
+    b = torch.zeros(N) if cfg.bias == "zero" else b[torch.arange(N) % 4].clone()
+    return e, b, [(i, j) for i in range(4) for j in range(i + 4, N, 4)]
+
+
+@pytest.mark.parametrize("name,T,K,mode", [("mid", 4096, None, "pairs"), ("mid", 333, 12, "groups"),
+                                           ("prefill", 8192, None, "pairs"), ("prefill", 1500, None, "groups"),
+                                           ("decode", 128, None, "pairs"), ("decode", 128, None, "groups")])
+def test_router_ties_and_order_through_the_fused_path(lib, name, T, K, mode):
+    """The fused router (tensor-core logits, cluster split, insertion lists
+    and butterfly merge) returns exactly the top-K of its own FP32 keys
+    fl32(s + b): ties go to the lower index and the list is ordered by key
+    descending, then index ascending. Checked bit for bit against the
+    oracle's top-K applied to the kernel's own affinities (scores_out), on
+    centroids with repeated rows so that equal keys really occur."""
+    import dataclasses
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    cfg = workloads.CONFIGS[name].with_tokens(T)
+    if K is not None:
+        cfg = dataclasses.replace(cfg, K_r=K)
+    u = workloads.activations(cfg)
+    e, b, tied = _tied_centroids(cfg, mode)
+    idx = torch.empty(cfg.T, cfg.K_r, dtype=torch.int32, device="cuda")
+    gates = torch.empty(cfg.T, cfg.K_r, dtype=torch.float32, device="cuda")
+    sc = torch.empty(cfg.T, cfg.N_r, dtype=torch.float32, device="cuda")
+    B.moe_route(u.cuda(), e.cuda(), b.cuda(), cfg.K_r, idx, gates, scores_out=sc)
+    torch.cuda.synchronize()
+    s_gpu = sc.cpu().double().numpy()
+    gi = idx.cpu().numpy().astype(np.int64)
+    bn = b.double().numpy()
+    # repeated centroid rows give bit-identical affinities
+    for lo, hi in tied:
+        assert np.array_equal(s_gpu[:, lo], s_gpu[:, hi]), (lo, hi)
+    # the selection and its order are the top-K of the kernel's own keys
+    ref = O.select_topk(s_gpu, bn, cfg.K_r)
+    bad = np.nonzero((gi != ref).any(axis=1))[0]
+    assert bad.size == 0, f"{bad.size} tokens differ, first {bad[:5]}: gpu {gi[bad[0]]} ref {ref[bad[0]]}"
+    # ties decided the selection somewhere: a tied partner left out at the
+    # K-th place, or two tied experts both selected
+    key = round_fp32(s_gpu + bn[None, :])
+    kth = np.take_along_axis(key, ref[:, -1:], axis=1)[:, 0]
+    outside = np.ones_like(key, dtype=bool)
+    np.put_along_axis(outside, ref, False, axis=1)
+    assert ((key == kth[:, None]) & outside).any(), "no tie at the selection boundary"
+    # gates are the selected affinities normalised in FP32
+    assert np.allclose(gates.cpu().double().numpy(), O.gates_from(s_gpu, ref), rtol=2e-6, atol=0)
+    # and the oracle's own routing agrees up to the 1e-5 margin rule
+    s64 = O.router_scores(u.double().numpy(), e.double().numpy())
+    assert np.abs(s_gpu - s64).max() < 1e-5
+    _check_routing(gi, s64, bn, cfg.K_r)
+
+
 # ---------------------------------------------------------------- permutation
 
 @pytest.mark.parametrize("T,N,K,pattern", [(1, 8, 2, "uniform"), (255, 8, 2, "uniform"),

@@ -1,13 +1,16 @@
 """End-to-end parity of the whole layer (MoELayerFP8 over the C ABI) with
-the CPU oracle on the five workloads.
+the CPU oracle on the five workloads, and on batches of 1 and 129 tokens.
 
-tiny and mid are compared on every token. prefill, decode and skew run at
+tiny, mid and decode are compared on every token. prefill and skew run at
 full size in the same launch configuration as the benchmark; the oracle
 routes all tokens (selection, counts, bias update) and computes the expert
-outputs for a seeded sample of tokens. Weights are drawn on the device by the
-seeded generator; the oracle receives the same FP32 weights copied to the
-host and quantises them itself (its codes and scales must equal the GPU's).
+outputs for 256 tokens: the first, the last, the 16 with the largest
+|u| (the outlier-heavy ones) and a seeded draw of the rest. Weights are drawn
+on the device by the seeded generator; the oracle receives the same FP32
+weights copied to the host and quantises them itself (its codes and scales
+must equal the GPU's).
 """
+import os
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -20,6 +23,17 @@ from tests.test_gpu_kernels import _check_routing, assert_close, f64
 
 pytestmark = pytest.mark.gpu
 
+SAMPLE = 256
+N_LARGEST = 16
+
+# The oracle's quantised weights of the last seed used, by slot: decode and
+# the T = 1 / T = 129 batches of the same layer share them.
+_QCACHE = {"key": None, "w": {}}
+
+
+def _threads():
+    return max(2, min(32, os.cpu_count() or 8))
+
 
 def _build(cfg, weights_on="cuda"):
     from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
@@ -30,7 +44,40 @@ def _build(cfg, weights_on="cuda"):
     return layer
 
 
-def _run(cfg, sample, weights_on):
+def _oracle_weights(cfg, slots, weights_on, ex):
+    """The oracle's own quantisation of the experts in `slots` (from the same
+    FP32 weights the layer received), a chunk of slots at a time."""
+    key = (cfg.seed, cfg.d, cfg.I, cfg.N_r, weights_on)
+    if _QCACHE["key"] != key:
+        _QCACHE["key"], _QCACHE["w"] = key, {}
+    cache = _QCACHE["w"]
+    todo = [s_ for s_ in slots if s_ not in cache]
+    quant = lambda h: O.quantise_expert(*[a.astype(np.float64) for a in h])
+    step = _threads()
+    for i in range(0, len(todo), step):
+        chunk = todo[i:i + step]
+        host = [[x.cpu().numpy() for x in workloads.expert_weights(cfg, s_, device=weights_on)]
+                for s_ in chunk]
+        cache.update(zip(chunk, ex.map(quant, host)))
+        del host
+    return {s_: cache[s_] for s_ in slots}
+
+
+def _sample(cfg, u, n=SAMPLE):
+    """Token sample: all tokens if there are at most n; else the first, the
+    last, the N_LARGEST tokens with the largest max |u|, and a seeded draw."""
+    T = cfg.T
+    if T <= n:
+        return np.arange(T)
+    big = np.argsort(-np.abs(u).max(axis=1), kind="stable")[:N_LARGEST]
+    fixed = np.unique(np.concatenate([[0, T - 1], big]))
+    rest = np.setdiff1d(np.arange(T), fixed)
+    rng = np.random.default_rng(cfg.seed + 17)
+    extra = rng.choice(rest, size=n - len(fixed), replace=False)
+    return np.sort(np.concatenate([fixed, extra]))
+
+
+def _run(cfg, weights_on, all_tokens=False):
     dev_inputs = cfg.T * cfg.d > 8_000_000
     gen_dev = "cuda" if dev_inputs else "cpu"
     u = workloads.activations(cfg, device=gen_dev)
@@ -44,6 +91,7 @@ def _run(cfg, sample, weights_on):
     assert B.moe_get_error() == 0
 
     un, en, bn = u.cpu().double().numpy(), e.cpu().double().numpy(), b.cpu().double().numpy()
+    sample = np.arange(cfg.T) if all_tokens else _sample(cfg, un)
     gpu_idx = layer.topk_idx.cpu().numpy().astype(np.int64)
     s64 = O.router_scores(un, en)
     diff = _check_routing(gpu_idx, s64, bn, cfg.K_r)
@@ -62,19 +110,15 @@ def _run(cfg, sample, weights_on):
     # oracle quantises the same FP32 weights itself (threads: numpy releases
     # the GIL), and its codes and scales must equal the GPU's
     slots = sorted(set(gpu_idx[sample].reshape(-1).tolist()) | {cfg.N_r})
-    host_w = {s_: [x.cpu().double().numpy() for x in workloads.expert_weights(cfg, s_, device=weights_on)]
-              for s_ in slots}
-    with ThreadPoolExecutor(max_workers=8) as ex:
-        quant = dict(zip(slots, ex.map(lambda s_: O.quantise_expert(*host_w[s_]), slots)))
-    del host_w
-    for s_, q in quant.items():
-        for key, t in [("gate_q", layer.w_gate), ("up_q", layer.w_up), ("down_q", layer.w_down)]:
-            assert np.array_equal(t[s_].cpu().numpy(), q[key]), (s_, key)
-        for key, t in [("gate_s", layer.s_gate), ("up_s", layer.s_up), ("down_s", layer.s_down)]:
-            assert np.array_equal(t[s_].cpu().double().numpy(), q[key]), (s_, key)
-    weights = quant.__getitem__
-
-    ref = O.moe_forward(un, en, bn, cfg.K_r, weights, tokens=sample, select=gpu_idx)
+    with ThreadPoolExecutor(max_workers=_threads()) as ex:
+        quant = _oracle_weights(cfg, slots, weights_on, ex)
+        for s_, q in quant.items():
+            for key, t in [("gate_q", layer.w_gate), ("up_q", layer.w_up), ("down_q", layer.w_down)]:
+                assert np.array_equal(t[s_].cpu().numpy(), q[key]), (s_, key)
+            for key, t in [("gate_s", layer.s_gate), ("up_s", layer.s_up), ("down_s", layer.s_down)]:
+                assert np.array_equal(t[s_].cpu().double().numpy(), q[key]), (s_, key)
+        ref = O.moe_forward(un, en, bn, cfg.K_r, quant.__getitem__, tokens=sample, select=gpu_idx,
+                            map_fn=ex.map)
     assert np.array_equal(layer.xq[torch.as_tensor(sample).cuda()].cpu().numpy(), ref["xq"])
     assert_close(f64(layer.y_shared)[sample], ref["y_shared"], "shared expert")
     yp = f64(layer.y_perm)
@@ -85,31 +129,36 @@ def _run(cfg, sample, weights_on):
     return layer
 
 
-def _sample(cfg, n, seed):
-    rng = np.random.default_rng(seed)
-    mid = rng.choice(np.arange(1, cfg.T - 1), size=min(n, cfg.T - 2), replace=False)
-    return np.unique(np.concatenate([[0, cfg.T - 1], mid]))
-
-
 def test_layer_tiny_all_tokens(lib):
     cfg = workloads.CONFIGS["tiny"]
-    _run(cfg, np.arange(cfg.T), weights_on="cpu")
+    _run(cfg, weights_on="cpu", all_tokens=True)
 
 
 def test_layer_tiny_ragged_tokens(lib):
     cfg = workloads.CONFIGS["tiny"].with_tokens(37)
-    _run(cfg, np.arange(cfg.T), weights_on="cpu")
+    _run(cfg, weights_on="cpu", all_tokens=True)
 
 
-def test_layer_mid_sampled(lib):
+def test_layer_mid_all_tokens(lib):
     cfg = workloads.CONFIGS["mid"]
-    _run(cfg, _sample(cfg, 62, seed=1), weights_on="cuda")
+    _run(cfg, weights_on="cuda", all_tokens=True)
 
 
-@pytest.mark.parametrize("name,n", [("decode", 6), ("prefill", 4), ("skew", 4)])
-def test_layer_full_size_sampled(lib, name, n):
+@pytest.mark.parametrize("T", [1, 129])
+def test_layer_mid_small_batches(lib, T):
+    # T = 1: one row per group and a one-row shared expert; T = 129: a
+    # ragged second row tile of the shared expert
+    _run(workloads.CONFIGS["mid"].with_tokens(T), weights_on="cuda", all_tokens=True)
+
+
+# decode and its 1- and 129-token batches run back to back (same weights)
+@pytest.mark.parametrize("name,T", [("decode", None), ("decode", 1), ("decode", 129),
+                                    ("prefill", None), ("skew", None)])
+def test_layer_full_size(lib, name, T):
     cfg = workloads.CONFIGS[name]
-    _run(cfg, _sample(cfg, n, seed=3), weights_on="cuda")
+    if T is not None:
+        cfg = cfg.with_tokens(T)
+    _run(cfg, weights_on="cuda")
 
 
 def test_layer_pipelined_host_path_matches_plain():
