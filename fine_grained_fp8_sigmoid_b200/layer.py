@@ -48,6 +48,17 @@ class MoELayerFP8:
         self.ws_gemm = torch.empty(max(B.moe_grouped_gemm_fp8_workspace(T, K_r, d, I), 256),
                                    dtype=u8, **dev)
 
+    def intermediate(self):
+        """Views of the last step's expert intermediate H in the GEMM
+        workspace (the layout include/moe_fp8.h gives for
+        moe_grouped_gemm_fp8): E4M3 codes [T*K_r + T][I] (routed rows in
+        permuted order, then the T shared rows) and their FP32 1x128 scales."""
+        rows, I = self.T * self.K_r + self.T, self.I
+        off = (rows * I + 255) // 256 * 256
+        codes = self.ws_gemm[:rows * I].view(rows, I)
+        scales = self.ws_gemm[off:off + rows * (I // 128) * 4].view(torch.float32).view(rows, I // 128)
+        return codes, scales
+
     # ---------------------------------------------------------------- weights
     def load_expert(self, slot: int, w_gate: torch.Tensor, w_up: torch.Tensor,
                     w_down: torch.Tensor, stream=None) -> None:

@@ -185,7 +185,10 @@ MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int K_r, int N_r
 /*
  * moe_grouped_gemm_fp8_workspace: bytes of scratch for the intermediate
  * H = requant(SwiGLU(...)) of P = T*K_r routed rows plus T shared rows:
- * (P + T) * I bytes of E4M3 and (P + T) * I/128 FP32 scales.
+ * (P + T) * I bytes of E4M3 and (P + T) * I/128 FP32 scales. After a call the
+ * workspace holds H: the codes [P + T][I] at its start (routed rows in
+ * xq_perm order, then the T shared rows), and the scales [P + T][I/128] from
+ * the next 256-byte boundary.
  */
 MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
 
@@ -215,7 +218,13 @@ MOE_API int moe_grouped_gemm_fp8_launches(int d, int I);
  *   w_gate, w_up      [N_r+1][I][d] E4M3;  s_gate, s_up  [N_r+1][I/128][d/128]
  *   w_down            [N_r+1][d][I] E4M3;  s_down        [N_r+1][d/128][I/128]
  *   y_perm            [P][d] FP32 (out)    y_shared [T][d] FP32 (out)
- *                     (FP32 so that h' is rounded to bf16 once, in moe_combine)
+ *                     FP32, not bf16: h' is rounded to bf16 once, in
+ *                     moe_combine. Rounding the expert outputs to bf16 as
+ *                     well puts outputs near a bf16 midpoint one ulp apart
+ *                     from the FP64 reference, which breaks the output
+ *                     tolerance where h' cancels to about zero; the cost is
+ *                     twice the output bytes (prefill: 2.11 GB written
+ *                     instead of 1.06 GB, and the same read by moe_combine).
  *   workspace         moe_grouped_gemm_fp8_workspace(T, K_r, d, I) bytes
  * Limits: d a multiple of 256, I a multiple of 128, N_r <= 1024.
  */

@@ -177,20 +177,32 @@ def silu(x: np.ndarray) -> np.ndarray:
         return x / (1.0 + np.exp(-x))
 
 
-def expert_ffn(xq, xs, w: dict):
-    """One expert on FP8 rows (xq, xs).
+def expert_ffn_parts(xq, xs, w: dict) -> dict:
+    """One expert on FP8 rows (xq, xs), with its intermediate values.
 
     a = silu(X W_gate^T) * (X W_up^T); a is rounded to FP32 (the precision
-    the kernel holds it in) and requantised per 1x128 tile along I; then
-    Y = H W_down^T, rounded to bf16 (the layer's output type).
-    Returns (Y bf16-rounded float64 [m, d], H dequantised float64 [m, I]).
+    the kernel holds it in) and requantised per 1x128 tile along I to
+    (hq, hs); then Y = H W_down^T, kept in float64 (the exact target of the
+    kernel's FP32 output).
+    Returns dict(a32 [m, I], hq uint8 [m, I], hs [m, I/128], y [m, d]).
     """
     G = scaled_gemm(xq, xs, w["gate_q"], w["gate_s"])
     U = scaled_gemm(xq, xs, w["up_q"], w["up_s"])
-    a = silu(G) * U
-    hq, hs = quant_1x128(round_fp32(a))
-    Y = scaled_gemm(hq, hs, w["down_q"], w["down_s"])
-    return Y, dequant_1x128(hq, hs)
+    a32 = round_fp32(silu(G) * U)
+    hq, hs = quant_1x128(a32)
+    return dict(a32=a32, hq=hq, hs=hs, y=expert_down(hq, hs, w))
+
+
+def expert_down(hq, hs, w: dict) -> np.ndarray:
+    """The down projection Y = H W_down^T of FP8 intermediate rows (hq, hs)."""
+    return scaled_gemm(hq, hs, w["down_q"], w["down_s"])
+
+
+def expert_ffn(xq, xs, w: dict):
+    """One expert on FP8 rows: returns (Y float64 [m, d], H dequantised
+    float64 [m, I]); see expert_ffn_parts."""
+    p = expert_ffn_parts(xq, xs, w)
+    return p["y"], dequant_1x128(p["hq"], p["hs"])
 
 
 # --------------------------------------------------------------------------
@@ -263,25 +275,30 @@ def moe_forward(u, e, b, K: int, weights, tokens=None, select=None, map_fn=map) 
     sample = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
     S = sample.shape[0]
     xq, xs = quant_1x128(u[sample])
-    y_routed = np.zeros((S, K, d))
-    h_routed = None
     sel = idx[sample]
     slots = [int(s_) for s_ in np.unique(sel)]
     whos = [np.argwhere(sel == slot) for slot in slots]      # rows (sample i, k)
 
     def one(j):
         if j == len(slots):
-            return expert_ffn(xq, xs, weights(N_r))
+            return expert_ffn_parts(xq, xs, weights(N_r))
         who = whos[j]
-        return expert_ffn(xq[who[:, 0]], xs[who[:, 0]], weights(slots[j]))
+        return expert_ffn_parts(xq[who[:, 0]], xs[who[:, 0]], weights(slots[j]))
 
     results = list(map_fn(one, range(len(slots) + 1)))
-    for who, (y, h) in zip(whos, results[:-1]):
-        if h_routed is None:
-            h_routed = np.zeros((S, K, h.shape[1]))
-        y_routed[who[:, 0], who[:, 1]] = y
-        h_routed[who[:, 0], who[:, 1]] = h
-    y_shared, h_shared = results[-1]
+    routed = {}
+    for who, p in zip(whos, results[:-1]):
+        for key, v in p.items():
+            if key not in routed:
+                routed[key] = np.zeros((S, K) + v.shape[1:], v.dtype)
+            routed[key][who[:, 0], who[:, 1]] = v
+    if not routed:
+        routed = dict(y=np.zeros((S, K, d)))
+    shared = results[-1]
+    y_routed, y_shared = routed["y"], shared["y"]
+    h_routed = (dequant_1x128(routed["hq"].reshape(S * K, -1), routed["hs"].reshape(S * K, -1)).reshape(S, K, -1)
+                if "hq" in routed else None)
+    h_shared = dequant_1x128(shared["hq"], shared["hs"])
 
     acc = u[sample] + y_shared
     for k in range(K):
@@ -291,4 +308,5 @@ def moe_forward(u, e, b, K: int, weights, tokens=None, select=None, map_fn=map) 
                 counts=counts, offsets=offsets, sorted_token=sorted_token,
                 inv=inv, bias_new=b_new, max_over_mean=ratio, tokens=sample,
                 xq=xq, xs=xs, y_routed=y_routed, h_routed=h_routed,
-                y_shared=y_shared, h_shared=h_shared, out=out)
+                y_shared=y_shared, h_shared=h_shared, out=out,
+                routed_parts=routed, shared_parts=shared)

@@ -15,25 +15,7 @@ from oracle.e4m3 import round_fp32
 
 pytestmark = pytest.mark.gpu
 
-RTOL, ATOL_RMS = 8e-3, 1e-3
-
-
-def f64(t):
-    return t.detach().to("cpu").double().numpy()
-
-
-def assert_close(gpu, ref, what):
-    gpu = np.asarray(gpu, np.float64)
-    ref = np.asarray(ref, np.float64)
-    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
-    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
-    err = np.abs(gpu - ref)
-    bound = RTOL * np.abs(ref) + ATOL_RMS * rms
-    bad = err > bound
-    if bad.any():
-        i = np.unravel_index(np.argmax(err - bound), err.shape)
-        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; "
-                             f"worst at {i}: gpu={gpu[i]} ref={ref[i]} rms={rms}")
+from tests.parity import assert_close, f64, near_tie_rows  # noqa: F401
 
 
 # ---------------------------------------------------------------- quantisers
@@ -338,13 +320,24 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
     torch.cuda.synchronize()
     assert B.moe_get_error() == 0
     yp = f64(y_perm)
-    for i in range(N_r):
-        a, b_ = offsets[i], offsets[i + 1]
-        if b_ > a:
-            ref, _ = O.expert_ffn(xq_p[a:b_], xs_p[a:b_], experts[i])
-            assert_close(yp[a:b_], ref, f"expert {i}")
-    ref, _ = O.expert_ffn(xq, xs, experts[N_r])
-    assert_close(f64(y_sh), ref, "shared expert")
+    rows = Ppad + T
+    hq_g = ws[:rows * I].view(rows, I).cpu().numpy()
+    off = (rows * I + 255) // 256 * 256
+    hs_g = ws[off:off + rows * (I // 128) * 4].view(torch.float32).view(rows, I // 128).cpu().double().numpy()
+    groups = [(i, offsets[i], offsets[i + 1], xq_p, xs_p) for i in range(N_r)] + [(N_r, 0, T, xq, xs)]
+    for i, a, b_, xq_i, xs_i in groups:
+        if b_ <= a:
+            continue
+        p = O.expert_ffn_parts(xq_i[a:b_], xs_i[a:b_], experts[i])
+        g0 = a if i < N_r else Ppad                 # the group's first row in H
+        flip, _ = near_tie_rows(hq_g[g0:g0 + b_ - a], hs_g[g0:g0 + b_ - a], p["a32"], p["hq"], p["hs"],
+                                f"expert {i} intermediate")
+        ref = p["y"]
+        if flip.size:
+            ref = ref.copy()
+            ref[flip] = O.expert_down(hq_g[g0 + flip], hs_g[g0 + flip], experts[i])
+        got = yp[a:b_] if i < N_r else f64(y_sh)
+        assert_close(got, ref, f"expert {i}")
 
 
 # ---------------------------------------------------------------- failure path
