@@ -34,8 +34,10 @@
 //            shared memory and TMA stores (the combine adds them to the
 //            residual and rounds once).
 // Tiles are numbered group-major (shared expert last), then row tile, then
-// column tile, and dealt round-robin to CTAs, so the CTAs running at the same
-// time share weight tiles and activation rows through L2.
+// column tile. The first wave is dealt by block index; after it each CTA
+// claims the next number from a counter in the workspace, so the tiles in
+// flight stay a window of about one wave and those sharing weight tiles and
+// activation rows read them from L2 at the same time.
 //
 // Narrow tiles: a group of only 1..64 rows (decode batches: a few tokens per
 // expert) would pay a 128 x 256 partial read-back per K block for them. Its
@@ -73,6 +75,7 @@ constexpr int EPI_WARP0 = 4;     // first epilogue warp
 constexpr uint32_t REGS_CTRL = 56;
 constexpr uint32_t REGS_EPI = 224;
 constexpr int MAX_GROUPS = 1025;
+constexpr int TILE_RING = 4;     // tile numbers the producer may publish ahead of the consumers
 constexpr uint32_t TMEM_COLS = 512;
 // narrow tiles: at most 64 token rows; K blocks of the tile's token-scale
 // table (phase 1: d/128, phase 2: I/128; phase 2 has less room beside the
@@ -105,6 +108,7 @@ struct Args {
   float* Hs;
   float* y_perm;
   float* y_shared;
+  int* tile_counter;         // zeroed before the launch; tiles past the first wave are claimed from it
 };
 
 template <int STAGES, int TAB_KB>
@@ -117,6 +121,9 @@ struct Smem {
   uint64_t xbar;      // epilogue exchange of max-abs partials (phase 1)
   uint64_t sbar;      // narrow tile: token-scale table staged (8 warps)
   uint64_t dbar;      // narrow tile: token-scale table no longer read (8 warps)
+  uint64_t rfull[TILE_RING];   // tile number published by the producer
+  uint64_t rfree[TILE_RING];   // read by the MMA thread and the 8 epilogue warps
+  int ring[TILE_RING];         // tile numbers in claim order; -1 ends the CTA's work
   uint32_t tmem_base;
   int abort;
   int total_tiles;
@@ -396,6 +403,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&sm.xbar, EPI_WARPS);
     mbar_init(&sm.sbar, EPI_WARPS);
     mbar_init(&sm.dbar, EPI_WARPS);
+    for (int i = 0; i < TILE_RING; ++i) {
+      mbar_init(&sm.rfull[i], 1);
+      mbar_init(&sm.rfree[i], 1 + EPI_WARPS);
+    }
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -451,8 +462,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       const uint64_t pol_w = l2_policy_evict_last();
-      for (int t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-        const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
+      // Dynamic schedule: the first wave takes tiles blockIdx.x, later tiles
+      // are claimed from a global counter when this CTA's previous tile has
+      // all its loads issued, so the CTAs stay within about one wave of each
+      // other and tiles that share weight blocks and activation rows run at
+      // the same time (their operands meet in L2). Each claimed number is
+      // published to the MMA thread and the epilogue through a ring in
+      // shared memory; -1 ends the CTA's work.
+      int rslot = 0;
+      uint32_t rph = 0;
+      int t = blockIdx.x;
+      for (;;) {
+        if (!mbar_wait(&sm.rfree[rslot], rph ^ 1, abort)) break;
+        const int tt = t < total ? t : -1;
+        sm.ring[rslot] = tt;
+        mbar_arrive(&sm.rfull[rslot]);
+        if (++rslot == TILE_RING) {
+          rslot = 0;
+          rph ^= 1;
+        }
+        if (tt < 0 || *abort) break;
+        const Tile tl = decode_tile<PHASE>(sm, a, tt, n_tiles);
         const CUtensorMap* am = (PHASE == 1 && tl.shared) ? &tm_x : &tm_a;
         const int arow = tl.row0 + tl.m * BM;
         for (int kb = 0; kb < KB; ++kb) {
@@ -474,6 +504,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             phase ^= 1;
           }
         }
+        t = static_cast<int>(gridDim.x) + atomicAdd(a.tile_counter, 1);
       }
       if (*abort) {
         volatile int never = 0;
@@ -488,7 +519,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       int buf = 0;
       uint32_t tphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      int rslot = 0;
+      uint32_t rph = 0;
+      while (ok) {
+        if (!mbar_wait(&sm.rfull[rslot], rph, abort)) break;
+        const int t = *reinterpret_cast<volatile int*>(&sm.ring[rslot]);
+        mbar_arrive(&sm.rfree[rslot]);
+        if (++rslot == TILE_RING) {
+          rslot = 0;
+          rph ^= 1;
+        }
+        if (t < 0) break;
         const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
         // narrow tile: the weights are M (two 128-row MMAs into columns 0 and
         // 128 of the buffer), the tile's first N = rows rounded up to 16 token
@@ -544,7 +585,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t xpar = 0;
     int n_narrow = 0;     // narrow tiles done (parity of sbar / dbar)
     const int KBd = a.d / BK, KBi = a.I / BK;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    int rslot = 0;
+    uint32_t rph = 0;
+    for (;;) {
+      if (!warp_wait(&sm.rfull[rslot], rph, abort)) break;
+      const int t = *reinterpret_cast<volatile int*>(&sm.ring[rslot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.rfree[rslot]);
+      if (++rslot == TILE_RING) {
+        rslot = 0;
+        rph ^= 1;
+      }
+      if (t < 0) break;
       const Tile tl = decode_tile<PHASE>(sm, a, t, n_tiles);
       if (tl.narrow) {
         NarrowCtx c{tmem + lane_base, q, half, lane, ew * 32 + lane, KB, abort};
@@ -589,33 +641,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!warp_wait(&sm.tfull[buf], tphase, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + lane_base + buf * BN;
-        float v[32];
-        if (PHASE == 1) {
-          const float fg = sa * s0, fu = sa * s1;
+        // four 32-column chunks of this thread's lane; the next chunk's read is
+        // in flight while the current one is scaled and accumulated, and the
+        // buffer is released as soon as the last chunk has arrived.
+        //   phase 1: gate columns half*64 + {0, 32}, then up columns 128 + half*64 + {0, 32}
+        //   phase 2: columns half*128 + {0, 32, 64, 96}
+        const uint32_t c0 = PHASE == 1 ? half * 64 : half * 128;
+        const uint32_t c2 = PHASE == 1 ? 128 + half * 64 : half * 128 + 64;
+        const float f01 = sa * s0, f23 = sa * s1;   // phase 2: s1 == s0
+        uint32_t ra[32], rb[32];
+        tmem_ld32_async(ta + c0, ra);
+        tmem_wait_ld(ra);
+        tmem_ld32_async(ta + c0 + 32, rb);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(ta + half * 64 + c * 32, v);
+        for (int j = 0; j < 32; ++j) acc[j] = fmaf(f01, __uint_as_float(ra[j]), acc[j]);
+        tmem_wait_ld(rb);
+        tmem_ld32_async(ta + c2, ra);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(fg, v[j], acc[c * 32 + j]);
-          }
+        for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(f01, __uint_as_float(rb[j]), acc[32 + j]);
+        tmem_wait_ld(ra);
+        tmem_ld32_async(ta + c2 + 32, rb);
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            tmem_ld32(ta + 128 + half * 64 + c * 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[64 + c * 32 + j] = fmaf(fu, v[j], acc[64 + c * 32 + j]);
-          }
-        } else {
-          const float f = sa * s0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(ta + half * 128 + c * 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(f, v[j], acc[c * 32 + j]);
-          }
-        }
+        for (int j = 0; j < 32; ++j) acc[64 + j] = fmaf(f23, __uint_as_float(ra[j]), acc[64 + j]);
+        tmem_wait_ld(rb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[96 + j] = fmaf(f23, __uint_as_float(rb[j]), acc[96 + j]);
         buf ^= 1;
         if (buf == 0) tphase ^= 1;
       }
@@ -721,11 +774,17 @@ inline int make_tmap_y(CUtensorMap* m, const float* base, uint64_t rows, uint64_
 }  // namespace gg
 }  // namespace moe
 
+// H codes, H scales (from the next 256-byte boundary), then two int32 tile
+// counters (one per launch, from the next 256-byte boundary)
+static size_t counters_offset(size_t rows, int I) {
+  return moe::gg::align256(moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float));
+}
+
 extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
   (void)d;
   if (T <= 0 || K_r <= 0 || I <= 0) return 0;
   const size_t rows = static_cast<size_t>(T) * K_r + T;
-  return moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float);
+  return counters_offset(rows, I) + 2 * sizeof(int);
 }
 
 // narrow tiles need the tile's [kb][token] activation-scale table to fit
@@ -778,9 +837,9 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   // Narrow tiles only when the average routed group has at most 64 rows
   // (decode-like batches). With larger groups the few small ones gain little
   // (an N <= 64 MMA costs about as much as an N = 256 one) and their slower
-  // tiles put the CTAs of the round-robin schedule out of step, so that tiles
-  // sharing weights and activation rows no longer meet in L2 (measured at
-  // T = 8192 with 39 groups of <= 64 rows: +4.2 GB of DRAM reads).
+  // tiles put the CTAs out of step, so that tiles sharing weights and
+  // activation rows no longer meet in L2 (measured with a static round-robin
+  // schedule at T = 8192 with 39 groups of <= 64 rows: +4.2 GB of DRAM reads).
   const bool narrow = narrow_enabled(d, I) && P <= static_cast<long long>(NMAX) * N_r;
 
   Args args;
@@ -800,6 +859,9 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   args.y_perm = y_perm;
   args.y_shared = y_shared;
   args.narrow_max = narrow ? NMAX : 0;
+  int* counters = reinterpret_cast<int*>(H + counters_offset(static_cast<size_t>(rowsH), I));
+  if (int st = cuda_status(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s), "grouped GEMM: tile counters"))
+    return st;
 
   // upper bound on row tiles: every non-empty routed group wastes < 1 tile
   const long long m_tiles = (P + BM - 1) / BM + (P < N_r ? P : N_r) + (T + BM - 1) / BM;
@@ -816,8 +878,10 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
                            "smem attribute (down)"))
     return st;
+  args.tile_counter = counters;
   k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
+  args.tile_counter = counters + 1;
   k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, args);
   if (int st = launch_status("grouped GEMM launch (down)")) return st;
   return MOE_OK;

@@ -188,7 +188,8 @@ MOE_API int moe_permute_noalloc(const int32_t* topk_idx, int T, int K_r, int N_r
  * (P + T) * I bytes of E4M3 and (P + T) * I/128 FP32 scales. After a call the
  * workspace holds H: the codes [P + T][I] at its start (routed rows in
  * xq_perm order, then the T shared rows), and the scales [P + T][I/128] from
- * the next 256-byte boundary.
+ * the next 256-byte boundary; after them (again 256-byte aligned) two int32
+ * tile counters, which each call zeroes on its stream before its launches.
  */
 MOE_API size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I);
 

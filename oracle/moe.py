@@ -184,13 +184,13 @@ def expert_ffn_parts(xq, xs, w: dict) -> dict:
     the kernel holds it in) and requantised per 1x128 tile along I to
     (hq, hs); then Y = H W_down^T, kept in float64 (the exact target of the
     kernel's FP32 output).
-    Returns dict(a32 [m, I], hq uint8 [m, I], hs [m, I/128], y [m, d]).
+    Returns dict(G, U, a32 [m, I], hq uint8 [m, I], hs [m, I/128], y [m, d]).
     """
     G = scaled_gemm(xq, xs, w["gate_q"], w["gate_s"])
     U = scaled_gemm(xq, xs, w["up_q"], w["up_s"])
     a32 = round_fp32(silu(G) * U)
     hq, hs = quant_1x128(a32)
-    return dict(a32=a32, hq=hq, hs=hs, y=expert_down(hq, hs, w))
+    return dict(G=G, U=U, a32=a32, hq=hq, hs=hs, y=expert_down(hq, hs, w))
 
 
 def expert_down(hq, hs, w: dict) -> np.ndarray:

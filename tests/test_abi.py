@@ -50,7 +50,9 @@ def test_workspace_sizes(lib):
     assert lib.moe_permute_workspace(0, 256) == 0
     rows = 8192 * 8 + 8192
     ws = lib.moe_grouped_gemm_fp8_workspace(8192, 8, 7168, 2048)
-    assert ws == ((rows * 2048 + 255) // 256) * 256 + rows * 16 * 4
+    a256 = lambda n: (n + 255) // 256 * 256
+    # H codes, H scales, two int32 tile counters, each part 256-byte aligned
+    assert ws == a256(a256(rows * 2048) + rows * 16 * 4) + 2 * 4
 
 
 def test_gemm_launch_count_query(lib):

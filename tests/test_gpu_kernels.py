@@ -15,7 +15,7 @@ from oracle.e4m3 import round_fp32
 
 pytestmark = pytest.mark.gpu
 
-from tests.parity import assert_close, f64, near_tie_rows  # noqa: F401
+from tests.parity import accumulation_bound, assert_close, f64, near_tie_rows  # noqa: F401
 
 
 # ---------------------------------------------------------------- quantisers
@@ -330,7 +330,8 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
             continue
         p = O.expert_ffn_parts(xq_i[a:b_], xs_i[a:b_], experts[i])
         g0 = a if i < N_r else Ppad                 # the group's first row in H
-        flip, _ = near_tie_rows(hq_g[g0:g0 + b_ - a], hs_g[g0:g0 + b_ - a], p["a32"], p["hq"], p["hs"],
+        da = accumulation_bound(xq_i[a:b_], xs_i[a:b_], experts[i], p["G"], p["U"])
+        flip, _ = near_tie_rows(hq_g[g0:g0 + b_ - a], hs_g[g0:g0 + b_ - a], p["a32"], da, p["hq"], p["hs"],
                                 f"expert {i} intermediate")
         ref = p["y"]
         if flip.size:

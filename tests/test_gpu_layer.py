@@ -19,7 +19,7 @@ import torch
 
 import workloads
 from oracle import moe as O
-from tests.parity import assert_close, f64, near_tie_rows
+from tests.parity import accumulation_bound, assert_close, f64, near_tie_rows
 from tests.test_gpu_kernels import _check_routing
 
 pytestmark = pytest.mark.gpu
@@ -134,13 +134,18 @@ def _run(cfg, weights_on, all_tokens=False):
     hs_g = np.concatenate([take(hs_all, rows_r), take(hs_all, rows_s)]).astype(np.float64)
     rp, sp = ref["routed_parts"], ref["shared_parts"]
     I = cfg.I
-    a32 = np.concatenate([rp["a32"].reshape(S * K, I), sp["a32"]])
-    hq_o = np.concatenate([rp["hq"].reshape(S * K, I), sp["hq"]])
-    hs_o = np.concatenate([rp["hs"].reshape(S * K, I // 128), sp["hs"]])
-    flip, dist = near_tie_rows(hq_g, hs_g, a32, hq_o, hs_o, f"{cfg.name} intermediate")
+    flat = lambda key, w: np.concatenate([rp[key].reshape(S * K, w), sp[key]])
+    a32, hq_o, hs_o = flat("a32", I), flat("hq", I), flat("hs", I // 128)
+    G, U = flat("G", I), flat("U", I)
+    slot_of = np.concatenate([gpu_idx[sample].reshape(-1), np.full(S, cfg.N_r)])
+    tok_of = np.concatenate([np.repeat(np.arange(S), K), np.arange(S)])   # row -> sample index
+    da = np.zeros_like(a32)
+    for s_ in np.unique(slot_of):
+        rr = np.nonzero(slot_of == s_)[0]
+        da[rr] = accumulation_bound(ref["xq"][tok_of[rr]], ref["xs"][tok_of[rr]], quant[int(s_)], G[rr], U[rr])
+    flip, dist = near_tie_rows(hq_g, hs_g, a32, da, hq_o, hs_o, f"{cfg.name} intermediate")
     y_r = ref["y_routed"].reshape(S * K, cfg.d).copy()
     y_s = ref["y_shared"].copy()
-    slot_of = np.concatenate([gpu_idx[sample].reshape(-1), np.full(S, cfg.N_r)])
     for s_ in np.unique(slot_of[flip]):
         rr = flip[slot_of[flip] == s_]
         y = O.expert_down(hq_g[rr], hs_g[rr], quant[int(s_)])
@@ -148,7 +153,7 @@ def _run(cfg, weights_on, all_tokens=False):
         y_r[rr[routed]] = y[routed]
         y_s[rr[~routed] - S * K] = y[~routed]
     print(f"[parity] {cfg.name} T={cfg.T}: {flip.size} of {hq_g.shape[0]} intermediate rows hold a "
-          f"near-tie code (max relative distance to the boundary {dist:.3g})")
+          f"near-tie code (max distance to the boundary {dist:.3g} of the bound)")
 
     assert_close(f64(layer.y_shared)[sample], y_s, "shared expert")
     yp = f64(layer.y_perm)

@@ -4,54 +4,65 @@ import numpy as np
 import pytest
 
 from oracle import moe as O
-from tests.parity import near_tie_rows
+from tests.parity import accumulation_bound, near_tie_rows
 
 
 def _case():
     rng = np.random.default_rng(5)
     a32 = np.float32(rng.standard_normal((4, 256))).astype(np.float64)
-    # a value whose x = a / scale sits on the boundary between 1.0 and 1.125
     hq, hs = O.quant_1x128(a32)
+    # x = a / scale just above the boundary between 1.0 and 1.125, and one
+    # far from every boundary
     a32[2, 7] = 1.0625 * hs[2, 0] * (1 + 1e-7)
-    a32[3, 9] = 1.03 * hs[3, 0]                  # far from every boundary
+    a32[3, 9] = 1.03 * hs[3, 0]
     hq, hs = O.quant_1x128(a32)
-    return a32, hq, hs
+    da = np.abs(a32) * 1e-6                    # a bound of one part in a million
+    return a32, da, hq, hs
 
 
 def test_identical_intermediate_has_no_near_ties():
-    a32, hq, hs = _case()
-    rows, dist = near_tie_rows(hq.copy(), hs.copy(), a32, hq, hs, "same")
+    a32, da, hq, hs = _case()
+    rows, dist = near_tie_rows(hq.copy(), hs.copy(), a32, da, hq, hs, "same")
     assert rows.size == 0 and dist == 0.0
 
 
-def test_adjacent_code_at_a_boundary_is_accepted():
-    a32, hq, hs = _case()
+def test_other_side_of_a_boundary_within_the_bound_is_accepted():
+    a32, da, hq, hs = _case()
     g = hq.copy()
-    assert g[2, 7] == 0x39                       # 1.125 (ties to the even mantissa)
-    g[2, 7] = 0x38                               # 1.0: the other side of the tie
-    rows, dist = near_tie_rows(g, hs, a32, hq, hs, "near tie")
-    assert list(rows) == [2] and dist < 1e-6
+    assert g[2, 7] == 0x39                       # 1.125
+    g[2, 7] = 0x38                               # 1.0: the other side of the boundary
+    rows, dist = near_tie_rows(g, hs, a32, da, hq, hs, "near tie")
+    assert list(rows) == [2] and dist < 1.0
 
 
-def test_code_change_away_from_a_boundary_is_rejected():
-    a32, hq, hs = _case()
-    g = hq.copy()
-    g[3, 9] += 1
-    with pytest.raises(AssertionError, match="away from a rounding boundary"):
-        near_tie_rows(g, hs, a32, hq, hs, "far")
-
-
-def test_code_two_steps_away_is_rejected():
-    a32, hq, hs = _case()
-    g = hq.copy()
-    g[2, 7] -= 2
-    with pytest.raises(AssertionError, match="more than one step"):
-        near_tie_rows(g, hs, a32, hq, hs, "two steps")
+def test_code_change_beyond_the_bound_is_rejected():
+    a32, da, hq, hs = _case()
+    for r, c, step in [(3, 9, 1), (2, 7, -2)]:
+        g = hq.copy()
+        g[r, c] = np.uint8(int(g[r, c]) + step)
+        with pytest.raises(AssertionError, match="outside the accumulation bound"):
+            near_tie_rows(g, hs, a32, da, hq, hs, "far")
 
 
 def test_scale_mismatch_is_rejected():
-    a32, hq, hs = _case()
+    a32, da, hq, hs = _case()
     s = hs.copy()
     s[1, 1] *= 1.001
     with pytest.raises(AssertionError, match="scale"):
-        near_tie_rows(hq, s, a32, hq, hs, "scale")
+        near_tie_rows(hq, s, a32, da, hq, hs, "scale")
+
+
+def test_accumulation_bound_grows_with_the_absolute_sums():
+    # one expert, two rows: the bound is proportional to sum |x w| and
+    # vanishes where U = 0 and silu(G) = 0
+    d = I = 128
+    xq = np.full((2, d), 0x38, np.uint8)
+    xs = np.array([[1.0], [2.0]])
+    w = dict(gate_q=np.full((I, d), 0x04, np.uint8), gate_s=np.ones((1, 1)),
+             up_q=np.full((I, d), 0x04, np.uint8), up_s=np.ones((1, 1)),
+             down_q=np.full((d, I), 0x04, np.uint8), down_s=np.ones((1, 1)))
+    p = O.expert_ffn_parts(xq, xs, w)
+    da = accumulation_bound(xq, xs, w, p["G"], p["U"])
+    assert np.all(da > 0) and np.all(da[1] > 2 * da[0])
+    zero = accumulation_bound(xq, xs, w, np.zeros((2, I)), np.zeros((2, I)))
+    assert np.all(zero == 0.0)
