@@ -76,6 +76,7 @@ constexpr uint32_t REGS_CTRL = 56;
 constexpr uint32_t REGS_EPI = 224;
 constexpr int MAX_GROUPS = 1025;
 constexpr int TILE_RING = 4;     // tile numbers the producer may publish ahead of the consumers
+constexpr int MMA_THREADS = 2;   // MMA issuers (lane 0 of warps 1 and 3): even and odd K blocks
 constexpr uint32_t TMEM_COLS = 512;
 // narrow tiles: at most 64 token rows; K blocks of the tile's token-scale
 // table (phase 1: d/128, phase 2: I/128; phase 2 has less room beside the
@@ -117,12 +118,12 @@ struct Smem {
   uint64_t empty[STAGES];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint64_t xbar;      // epilogue exchange of max-abs partials (phase 1)
   uint64_t sbar;      // narrow tile: token-scale table staged (8 warps)
   uint64_t dbar;      // narrow tile: token-scale table no longer read (8 warps)
   uint64_t rfull[TILE_RING];   // tile number published by the producer
-  uint64_t rfree[TILE_RING];   // read by the MMA thread and the 8 epilogue warps
+  uint64_t rfree[TILE_RING];   // read by the 2 MMA threads and the 8 epilogue warps
   int ring[TILE_RING];         // tile numbers in claim order; -1 ends the CTA's work
   uint32_t tmem_base;
   int abort;
@@ -399,13 +400,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&sm.tfull[b], 1);
       mbar_init(&sm.tempty[b], EPI_WARPS);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain[0], 1);
+    mbar_init(&sm.drain[1], 1);
     mbar_init(&sm.xbar, EPI_WARPS);
     mbar_init(&sm.sbar, EPI_WARPS);
     mbar_init(&sm.dbar, EPI_WARPS);
     for (int i = 0; i < TILE_RING; ++i) {
       mbar_init(&sm.rfull[i], 1);
-      mbar_init(&sm.rfree[i], 1 + EPI_WARPS);
+      mbar_init(&sm.rfree[i], MMA_THREADS + EPI_WARPS);
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -511,13 +513,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int s = 0; s < STAGES; ++s)
           if (armed[s] >= 0) mbar_wait(&sm.full[s], armed[s], &never, 100000000ull);
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------ MMA issuer
+    } else if ((warp == 1 || warp == 3) && lane == 0) {
+      // ------------------------------------------------ MMA issuers
+      // Issuing a K block's four MMAs and two commits, after two barrier
+      // checks, is a chain of long-latency instructions for one thread
+      // (about a microsecond's worth of issue latency next to the epilogue's
+      // FMA streams, measured). Two threads on different SM sub-partitions
+      // take alternate K blocks of the CTA's sequence: thread j the blocks
+      // k = j (mod 2), which use TMEM buffer j and every other pipeline stage,
+      // so their chains overlap while each buffer is still filled and drained
+      // in order.
+      const int j = warp == 1 ? 0 : 1;
       const uint32_t idesc = make_idesc(0, 0, BM, BN);
-      int stage = 0;
+      int stage = j;              // stage of this thread's next K block
       uint32_t phase = 0;
-      int buf = 0;
+      const int buf = j;
       uint32_t tphase = 0;
+      uint32_t kpar = 0;          // parity of the CTA's K-block sequence
       bool ok = true;
       int rslot = 0;
       uint32_t rph = 0;
@@ -535,9 +547,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 128 of the buffer), the tile's first N = rows rounded up to 16 token
         // rows of the A stage are N
         const uint32_t idesc_n = make_idesc(0, 0, 128, (tl.mrows + 15) & ~15);
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) { ok = false; break; }
+        for (int kb = 0; kb < KB; ++kb, kpar ^= 1) {
+          if (kpar != static_cast<uint32_t>(j)) continue;
+          // the operands usually land well before the partial buffer is free:
+          // check them first, so that only the buffer's wait sits between the
+          // epilogue's release and the next MMAs
           if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
+          if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
           const uint64_t ad = sw128_kmajor_desc(a_addr);
@@ -547,9 +563,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) umma_f8f6f4(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0);
           } else {
-            // the two accumulators' K steps interleaved: an MMA costs about
-            // the same for N <= 64 as for N = 256, and two independent chains
-            // overlap in the tensor pipe where one dependent chain does not
+            // the two accumulators' K steps interleaved (independent chains
+            // overlap in the tensor pipe)
             const uint64_t wd0 = sw128_kmajor_desc(a_addr + A_BYTES);
             const uint64_t wd1 = sw128_kmajor_desc(a_addr + A_BYTES + B_BYTES / 2);
 #pragma unroll
@@ -560,17 +575,17 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           umma_commit(&sm.empty[stage]);
           umma_commit(&sm.tfull[buf]);
-          if (++stage == STAGES) {
-            stage = 0;
+          stage += 2;                 // this thread's next block is two ahead
+          if (stage >= STAGES) {
+            stage -= STAGES;
             phase ^= 1;
           }
-          buf ^= 1;
-          if (buf == 0) tphase ^= 1;
+          tphase ^= 1;
         }
       }
-      umma_commit(&sm.drain);
+      umma_commit(&sm.drain[j]);
       volatile int never = 0;
-      mbar_wait(&sm.drain, 0, &never, 100000000ull);
+      mbar_wait(&sm.drain[j], 0, &never, 100000000ull);
     }
   } else {
     // ------------------------------------------------ epilogue
@@ -641,9 +656,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!warp_wait(&sm.tfull[buf], tphase, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ta = tmem + lane_base + buf * BN;
-        // four 32-column chunks of this thread's lane; the next chunk's read is
-        // in flight while the current one is scaled and accumulated, and the
-        // buffer is released as soon as the last chunk has arrived.
+        // four 32-column chunks of this thread's lane, read two at a time: the
+        // first two land together; the third and fourth are issued as soon as
+        // the registers of the first and second are consumed, and the buffer
+        // is released when they have landed (two read latencies and two chunks
+        // of FMAs after the buffer became full).
         //   phase 1: gate columns half*64 + {0, 32}, then up columns 128 + half*64 + {0, 32}
         //   phase 2: columns half*128 + {0, 32, 64, 96}
         const uint32_t c0 = PHASE == 1 ? half * 64 : half * 128;
@@ -651,22 +668,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float f01 = sa * s0, f23 = sa * s1;   // phase 2: s1 == s0
         uint32_t ra[32], rb[32];
         tmem_ld32_async(ta + c0, ra);
-        tmem_wait_ld(ra);
         tmem_ld32_async(ta + c0 + 32, rb);
+        tmem_wait_ld(ra);
+        tmem_wait_ld(rb);
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[j] = fmaf(f01, __uint_as_float(ra[j]), acc[j]);
-        tmem_wait_ld(rb);
         tmem_ld32_async(ta + c2, ra);
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(f01, __uint_as_float(rb[j]), acc[32 + j]);
-        tmem_wait_ld(ra);
         tmem_ld32_async(ta + c2 + 32, rb);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[64 + j] = fmaf(f23, __uint_as_float(ra[j]), acc[64 + j]);
+        tmem_wait_ld(ra);
         tmem_wait_ld(rb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[64 + j] = fmaf(f23, __uint_as_float(ra[j]), acc[64 + j]);
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[96 + j] = fmaf(f23, __uint_as_float(rb[j]), acc[96 + j]);
         buf ^= 1;
