@@ -478,6 +478,7 @@ def run_ours(args, rank, world, local_rank):
     b = b0.clone()
     torch.cuda.synchronize(dev)
     gemm_launches = B.moe_grouped_gemm_fp8_launches(cfg.d, cfg.I)
+    launches_per_step = layer.launches_per_step()
     K = args.steps
     ms_step, gemm_ms, clocks = time_layer(layer, u, e, b, K, args.warmup, dev, world, local_rank)
     tokens_per_s = whole_job_tokens_per_s(cfg.T, world, ms_step)
@@ -527,9 +528,9 @@ def run_ours(args, rank, world, local_rank):
                              traffic=gemm_traffic(cfg)),
             "cpu_baseline": cpu,
             "e2e": e2e,
-            # quant, router, permute (count, scan, scatter, gather), the GEMM's
-            # launches, combine, bias update
-            "gpu_launches": (8 + gemm_launches) * K,
+            # router, quant, permute (count, scan, scatter, and the row gather
+            # unless fused into the GEMM), the GEMM's launches, combine, bias update
+            "gpu_launches": launches_per_step * K,
             "balance": balance,
             "clocks": clocks,
         }

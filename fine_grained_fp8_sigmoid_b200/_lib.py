@@ -34,6 +34,8 @@ SIGNATURES = {
     "moe_grouped_gemm_fp8_launches": (_i, [_i, _i]),
     "moe_grouped_gemm_fp8": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p,
                                   _i, _i, _p, _p, _p, _z, _p]),
+    "moe_grouped_gemm_fp8_gather": (_i, [_p, _p, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p,
+                                         _i, _i, _p, _p, _p, _z, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _p, _i, _i, _i, _f, _p, _p]),
     "moe_debug_wait_timeout": (_i, [_i, _p]),

@@ -165,6 +165,35 @@ def moe_grouped_gemm_fp8(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_grouped_gemm_fp8_gather(sorted_token, offsets, xq, xs, w_gate, w_up, w_down,
+                                s_gate, s_up, s_down, y_perm, y_shared, workspace, stream=None):
+    """moe_grouped_gemm_fp8 with the routed rows read from xq/xs at sorted_token."""
+    T, d = xq.shape
+    P = sorted_token.shape[0]
+    G, I, _ = w_gate.shape
+    N_r = G - 1
+    K_r = P // T if T else 0
+    _want(sorted_token, torch.int32, (P,), "sorted_token")
+    _want(offsets, torch.int32, (N_r + 1,), "offsets")
+    _want(xq, torch.uint8, (T, d), "xq")
+    _want(xs, torch.float32, (T, d // 128), "xs")
+    _want(w_gate, torch.uint8, (G, I, d), "w_gate")
+    _want(w_up, torch.uint8, (G, I, d), "w_up")
+    _want(w_down, torch.uint8, (G, d, I), "w_down")
+    _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
+    _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
+    _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
+    _want(y_perm, torch.float32, (P, d), "y_perm")
+    _want(y_shared, torch.float32, (T, d), "y_shared")
+    if T and P != T * K_r:
+        raise ValueError("sorted_token must hold T * K_r rows")
+    check("moe_grouped_gemm_fp8_gather", _lib.load().moe_grouped_gemm_fp8_gather(
+        _ptr(sorted_token), _ptr(offsets), N_r, K_r, _ptr(xq), _ptr(xs), T,
+        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(s_gate), _ptr(s_up), _ptr(s_down),
+        d, I, _ptr(y_perm), _ptr(y_shared), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
     T, d = u.shape
     K_r = inv.shape[1]

@@ -110,6 +110,7 @@ struct Args {
   float* y_perm;
   float* y_shared;
   int* tile_counter;         // zeroed before the launch; tiles past the first wave are claimed from it
+  const int32_t* sorted_token;  // non-null: routed rows are read from xq/xs at these tokens (no xq_perm)
 };
 
 template <int STAGES, int TAB_KB>
@@ -197,6 +198,20 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* s
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
+// Four rows y0..y3 of a 2-D tensor (box: one row of 128 bytes) into four
+// consecutive 128-byte rows of shared memory, completion counted on `bar`.
+// The tensor map's 128-byte swizzle is applied by shared-memory address, so
+// four such loads at 512-byte steps from a 1024-byte aligned base lay out 16
+// rows exactly as one 16-row tile load would.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until at most N bulk groups of this thread still read shared memory
 template <int N>
@@ -250,11 +265,16 @@ __device__ __forceinline__ bool narrow_tile(S& sm, const Args& a, const Tile tl,
   // stage the table once the previous narrow tile's table is read by all warps
   if (nn > 0 && !warp_wait(&sm.dbar, (nn - 1) & 1, x.abort)) return false;
   {
+    const bool gathered = PHASE == 1 && !tl.shared && a.sorted_token != nullptr;
     const float* xsrc = PHASE == 1 ? (tl.shared ? a.xs : a.xs_perm) + static_cast<size_t>(r0) * KBd
                                    : a.Hs + static_cast<size_t>(r0) * KBi;
     for (int e = x.tid; e < x.KB * NMAX; e += EPI_THREADS) {
       const int kb = e / NMAX, j = e % NMAX;
-      sm.xs_tab[kb][j] = j < tl.mrows ? __ldg(xsrc + static_cast<size_t>(j) * x.KB + kb) : 0.0f;
+      float v = 0.0f;
+      if (j < tl.mrows)
+        v = gathered ? __ldg(a.xs + static_cast<size_t>(__ldg(a.sorted_token + r0 + j)) * KBd + kb)
+                     : __ldg(xsrc + static_cast<size_t>(j) * x.KB + kb);
+      sm.xs_tab[kb][j] = v;
     }
   }
   __syncwarp();
@@ -376,7 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
                         const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_ys,
-                        const Args a) {
+                        const __grid_constant__ CUtensorMap tm_xg, const Args a) {
   constexpr int STAGES = Cfg<PHASE>::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -417,6 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_b0);
     tma_prefetch_desc(&tm_b1);
+    if (PHASE == 1 && a.sorted_token != nullptr) tma_prefetch_desc(&tm_xg);
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
@@ -457,8 +478,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp < EPI_WARP0) {
     regs_decrease<REGS_CTRL>();
-    if (warp == 0 && lane == 0) {
+    if (warp == 0) {
       // ------------------------------------------------ TMA producer
+      // Lane 0 owns the barriers and the schedule. When the routed rows are
+      // gathered from xq (sorted_token given), every lane also issues one
+      // four-row gather per K block: lane i fetches rows 4i..4i+3 of the A tile.
       int armed[STAGES];
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
       int stage = 0;
@@ -469,50 +493,80 @@ __global__ void __launch_bounds__(THREADS, 1)
       // all its loads issued, so the CTAs stay within about one wave of each
       // other and tiles that share weight blocks and activation rows run at
       // the same time (their operands meet in L2). Each claimed number is
-      // published to the MMA thread and the epilogue through a ring in
+      // published to the MMA threads and the epilogue through a ring in
       // shared memory; -1 ends the CTA's work.
       int rslot = 0;
       uint32_t rph = 0;
       int t = blockIdx.x;
       for (;;) {
-        if (!mbar_wait(&sm.rfree[rslot], rph ^ 1, abort)) break;
-        const int tt = t < total ? t : -1;
-        sm.ring[rslot] = tt;
-        mbar_arrive(&sm.rfull[rslot]);
-        if (++rslot == TILE_RING) {
-          rslot = 0;
-          rph ^= 1;
+        int tt = -1, okr = 1;
+        if (lane == 0) {
+          okr = mbar_wait(&sm.rfree[rslot], rph ^ 1, abort) ? 1 : 0;
+          if (okr) {
+            tt = t < total ? t : -1;
+            sm.ring[rslot] = tt;
+            mbar_arrive(&sm.rfull[rslot]);
+            if (++rslot == TILE_RING) {
+              rslot = 0;
+              rph ^= 1;
+            }
+          }
         }
-        if (tt < 0 || *abort) break;
+        okr = __shfl_sync(0xffffffffu, okr, 0);
+        tt = __shfl_sync(0xffffffffu, tt, 0);
+        if (!okr || tt < 0 || *abort) break;
         const Tile tl = decode_tile<PHASE>(sm, a, tt, n_tiles);
+        const bool gather = PHASE == 1 && !tl.shared && a.sorted_token != nullptr;
         const CUtensorMap* am = (PHASE == 1 && tl.shared) ? &tm_x : &tm_a;
         const int arow = tl.row0 + tl.m * BM;
+        int tok[4] = {0, 0, 0, 0};
+        // gathered tiles fetch only the four-row groups holding rows of the
+        // group (the tile's other rows keep stale data; their products are
+        // never stored)
+        const int live = gather ? min(BM, tl.rows - tl.m * BM) : 0;
+        const int n_g4 = (live + 3) / 4;
+        if (gather && lane < n_g4) {
+          const int last = tl.row0 + tl.rows - 1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tok[i] = __ldg(a.sorted_token + min(arow + 4 * lane + i, last));
+        }
+        const uint32_t stage_bytes = gather ? STAGE_BYTES - A_BYTES + n_g4 * 4 * BK : STAGE_BYTES;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&sm.empty[stage], phase ^ 1, abort)) break;
+          int okw = 1;
           uint8_t* dst = tiles + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&sm.full[stage], STAGE_BYTES);
-          tma_load_2d(dst, am, &sm.full[stage], kb * BK, arow);
-          if (PHASE == 1) {
-            const int wrow = tl.g * a.I + tl.n * 128;
-            tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
-            tma_load_2d_hint(dst + A_BYTES + B_BYTES / 2, &tm_b1, &sm.full[stage], kb * BK, wrow, pol_w);
-          } else {
-            const int wrow = tl.g * a.d + tl.n * BN;
-            tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+          if (lane == 0) {
+            okw = mbar_wait(&sm.empty[stage], phase ^ 1, abort) ? 1 : 0;
+            if (okw) {
+              mbar_arrive_expect_tx(&sm.full[stage], stage_bytes);
+              if (!gather) tma_load_2d(dst, am, &sm.full[stage], kb * BK, arow);
+              if (PHASE == 1) {
+                const int wrow = tl.g * a.I + tl.n * 128;
+                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+                tma_load_2d_hint(dst + A_BYTES + B_BYTES / 2, &tm_b1, &sm.full[stage], kb * BK, wrow, pol_w);
+              } else {
+                const int wrow = tl.g * a.d + tl.n * BN;
+                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+              }
+              armed[stage] = phase;
+            }
           }
-          armed[stage] = phase;
+          okw = __shfl_sync(0xffffffffu, okw, 0);   // also orders the copies after the expected bytes
+          if (!okw) break;
+          if (gather && lane < n_g4)
+            tma_gather4(dst + lane * 4 * BK, &tm_xg, &sm.full[stage], kb * BK, tok[0], tok[1], tok[2], tok[3]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        t = static_cast<int>(gridDim.x) + atomicAdd(a.tile_counter, 1);
+        if (lane == 0) t = static_cast<int>(gridDim.x) + atomicAdd(a.tile_counter, 1);
       }
-      if (*abort) {
+      if (lane == 0 && *abort) {
         volatile int never = 0;
         for (int s = 0; s < STAGES; ++s)
           if (armed[s] >= 0) mbar_wait(&sm.full[s], armed[s], &never, 100000000ull);
       }
+      __syncwarp();
     } else if ((warp == 1 || warp == 3) && lane == 0) {
       // ------------------------------------------------ MMA issuers
       // Issuing a K block's four MMAs and two commits, after two barrier
@@ -632,7 +686,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float* sb0;
       const float* sb1;
       if (PHASE == 1) {
-        sa_ptr = (tl.shared ? a.xs : a.xs_perm) + static_cast<size_t>(grow) * KBd;
+        if (tl.shared || a.sorted_token == nullptr)
+          sa_ptr = (tl.shared ? a.xs : a.xs_perm) + static_cast<size_t>(grow) * KBd;
+        else   // gathered rows: the scales of the row's token
+          sa_ptr = a.xs + static_cast<size_t>(valid ? __ldg(a.sorted_token + grow) : 0) * KBd;
         sb0 = a.s_gate + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
         sb1 = a.s_up + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
       } else {
@@ -815,12 +872,13 @@ extern "C" int moe_grouped_gemm_fp8_launches(int d, int I) {
   return 2;
 }
 
-extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
-                                    int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
-                                    const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
-                                    const float* s_gate, const float* s_up, const float* s_down, int d,
-                                    int I, float* y_perm, float* y_shared, void* workspace,
-                                    size_t ws_bytes, void* stream) {
+// Both entry points: the routed rows come from xq_perm/xs_perm, or (sorted_token
+// non-null) straight from xq/xs at the tokens sorted_token lists.
+static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int32_t* sorted_token,
+                        const int32_t* offsets, int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
+                        const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down, const float* s_gate,
+                        const float* s_up, const float* s_down, int d, int I, float* y_perm, float* y_shared,
+                        void* workspace, size_t ws_bytes, void* stream) {
   using namespace moe;
   using namespace moe::gg;
   MOE_CHECK_ARG(N_r >= 1 && K_r >= 1 && T >= 0 && d > 0 && I > 0);
@@ -828,8 +886,9 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   const long long P = static_cast<long long>(T) * K_r;
   MOE_CHECK_SUPPORTED(P + T < (1LL << 31) && static_cast<long long>(N_r + 1) * (d > I ? d : I) < (1LL << 31));
   if (T == 0) return MOE_OK;
-  MOE_CHECK_ARG(xq_perm && xs_perm && offsets && xq && xs && w_gate && w_up && w_down && s_gate && s_up &&
-                s_down && y_perm && y_shared && workspace);
+  const bool gather = sorted_token != nullptr;
+  MOE_CHECK_ARG((gather || (xq_perm && xs_perm)) && offsets && xq && xs && w_gate && w_up && w_down && s_gate &&
+                s_up && s_down && y_perm && y_shared && workspace);
   MOE_CHECK_ARG(ws_bytes >= moe_grouped_gemm_fp8_workspace(T, K_r, d, I));
   MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(workspace) % 256 == 0 && reinterpret_cast<uintptr_t>(y_perm) % 16 == 0 &&
                 reinterpret_cast<uintptr_t>(y_shared) % 16 == 0);
@@ -841,10 +900,17 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   uint8_t* H = static_cast<uint8_t*>(workspace);
   float* Hs = reinterpret_cast<float*>(H + align256(static_cast<size_t>(rowsH) * I));
 
-  CUtensorMap tmA, tmX, tmWg, tmWu, tmH, tmWd, tmY, tmYs;
+  CUtensorMap tmA, tmX, tmXg, tmWg, tmWu, tmH, tmWd, tmY, tmYs;
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  if (int st = make_tmap_2d(&tmA, xq_perm, U8, 1, P, d, BM, BK)) return st;
   if (int st = make_tmap_2d(&tmX, xq, U8, 1, T, d, BM, BK)) return st;
+  if (gather) {
+    // one-row boxes of xq for the four-row gathers; tmA is then unused
+    if (int st = make_tmap_2d(&tmXg, xq, U8, 1, T, d, 1, BK)) return st;
+    tmA = tmX;
+  } else {
+    if (int st = make_tmap_2d(&tmA, xq_perm, U8, 1, P, d, BM, BK)) return st;
+    tmXg = tmX;
+  }
   if (int st = make_tmap_2d(&tmWg, w_gate, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
   if (int st = make_tmap_2d(&tmWu, w_up, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
   if (int st = make_tmap_2d(&tmH, H, U8, 1, rowsH, I, BM, BK)) return st;
@@ -876,6 +942,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
   args.y_perm = y_perm;
   args.y_shared = y_shared;
   args.narrow_max = narrow ? NMAX : 0;
+  args.sorted_token = sorted_token;
   int* counters = reinterpret_cast<int*>(H + counters_offset(static_cast<size_t>(rowsH), I));
   if (int st = cuda_status(cudaMemsetAsync(counters, 0, 2 * sizeof(int), s), "grouped GEMM: tile counters"))
     return st;
@@ -896,10 +963,30 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
                            "smem attribute (down)"))
     return st;
   args.tile_counter = counters;
-  k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, args);
+  k1<<<g1, THREADS, sm1, s>>>(tmA, tmX, tmWg, tmWu, tmY, tmYs, tmXg, args);
   if (int st = launch_status("grouped GEMM launch (gate/up)")) return st;
   args.tile_counter = counters + 1;
-  k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, args);
+  k2<<<g2, THREADS, sm2, s>>>(tmH, tmH, tmWd, tmWd, tmY, tmYs, tmXg, args);
   if (int st = launch_status("grouped GEMM launch (down)")) return st;
   return MOE_OK;
+}
+
+extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
+                                    int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
+                                    const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
+                                    const float* s_gate, const float* s_up, const float* s_down, int d,
+                                    int I, float* y_perm, float* y_shared, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_r, K_r, xq, xs, T, w_gate, w_up, w_down, s_gate, s_up,
+                      s_down, d, I, y_perm, y_shared, workspace, ws_bytes, stream);
+}
+
+extern "C" int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token, const int32_t* offsets, int N_r, int K_r,
+                                           const uint8_t* xq, const float* xs, int T, const uint8_t* w_gate,
+                                           const uint8_t* w_up, const uint8_t* w_down, const float* s_gate,
+                                           const float* s_up, const float* s_down, int d, int I, float* y_perm,
+                                           float* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+  // a null sorted_token falls to the materialised-rows check (INVALID_ARG)
+  return grouped_gemm(nullptr, nullptr, sorted_token, offsets, N_r, K_r, xq, xs, T, w_gate, w_up, w_down, s_gate,
+                      s_up, s_down, d, I, y_perm, y_shared, workspace, ws_bytes, stream);
 }

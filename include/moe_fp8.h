@@ -239,6 +239,26 @@ MOE_API int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_grouped_gemm_fp8_gather: moe_grouped_gemm_fp8 with the permutation's row
+ * movement fused into the GEMM's loads: the routed rows are read from xq/xs
+ * at the tokens sorted_token lists (moe_permute called with xq = NULL), so
+ * xq_perm and xs_perm are never written or read. Same products, scales,
+ * outputs, workspace and limits as moe_grouped_gemm_fp8 (the FP8 operands of
+ * each row are the same bytes, so the outputs are bit-identical to it).
+ *   sorted_token  [T*K_r] int32 (device) from moe_permute; values in [0, T)
+ * The A tiles of routed rows arrive as four-row TMA gathers of xq, one per
+ * lane of the producer warp per K block.
+ */
+MOE_API int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token,
+                         const int32_t* offsets, int N_r, int K_r,
+                         const uint8_t* xq, const float* xs, int T,
+                         const uint8_t* w_gate, const uint8_t* w_up,
+                         const uint8_t* w_down, const float* s_gate,
+                         const float* s_up, const float* s_down, int d, int I,
+                         float* y_perm, float* y_shared,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
  * ("DeepSeek-V3 Teknik Raporu", Yöntem 2, the h'_t equation). The sum is FP32
  * in the fixed order u, shared, k = 0..K_r-1.

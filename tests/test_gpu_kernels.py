@@ -341,6 +341,72 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
         assert_close(got, ref, f"expert {i}")
 
 
+@pytest.mark.parametrize("d,I,T,K,N_r", [(512, 256, 300, 3, 7), (2048, 1024, 700, 6, 16),
+                                         (7168, 2048, 200, 8, 12),
+                                         # average group <= 64 rows: narrow tiles
+                                         (512, 256, 90, 4, 16)])
+def test_grouped_gemm_gather_matches_materialised(lib, d, I, T, K, N_r):
+    """moe_grouped_gemm_fp8_gather (routed rows gathered from xq by the GEMM's
+    loads) gives bit for bit what moe_grouped_gemm_fp8 gives on the
+    materialised xq_perm, intermediate included, and matches the oracle."""
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    rng = np.random.default_rng(d + T)
+    x = round_fp32(rng.standard_normal((T, d)) * np.exp2(rng.integers(-3, 3, (T, 1))))
+    xq, xs = O.quant_1x128(x)
+    idx = workloads.topk_indices(T, N_r, K, seed=T + K).numpy()
+    counts, offsets, sorted_token, _ = O.permute(idx, N_r)
+    experts = []
+    for _ in range(N_r + 1):
+        w = [round_fp32(rng.standard_normal(sh) * 0.02) for sh in [(I, d), (I, d), (d, I)]]
+        experts.append(O.quantise_expert(*w))
+    dev = dict(device="cuda")
+    cu = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
+    P = T * K
+    stack = lambda key, dt: cu(np.stack([e[key] for e in experts]), dt)
+    W = [stack(k, torch.uint8) for k in ("gate_q", "up_q", "down_q")] + \
+        [stack(k, torch.float32) for k in ("gate_s", "up_s", "down_s")]
+    xq_d, xs_d = cu(xq, torch.uint8), cu(xs, torch.float32)
+    st_d, off_d = cu(sorted_token, torch.int32), cu(offsets, torch.int32)
+    outs = []
+    for gathered in (False, True):
+        y_perm = torch.full((P, d), float("nan"), dtype=torch.float32, **dev)
+        y_sh = torch.full((T, d), float("nan"), dtype=torch.float32, **dev)
+        ws = torch.zeros(B.moe_grouped_gemm_fp8_workspace(T, K, d, I), dtype=torch.uint8, **dev)
+        if gathered:
+            B.moe_grouped_gemm_fp8_gather(st_d, off_d, xq_d, xs_d, *W, y_perm, y_sh, ws)
+        else:
+            B.moe_grouped_gemm_fp8(xq_d[st_d.long()].contiguous(), xs_d[st_d.long()].contiguous(), off_d,
+                                   xq_d, xs_d, *W, y_perm, y_sh, ws)
+        torch.cuda.synchronize()
+        assert B.moe_get_error() == 0
+        rows = P + T
+        outs.append((y_perm.cpu(), y_sh.cpu(), ws[:rows * I].cpu()))
+    for a_, b_ in zip(*outs):
+        assert torch.equal(a_, b_)
+    # and the oracle, on every routed group and the shared expert, under the
+    # intermediate's near-tie rule (tests/parity.py)
+    yp, ysh = outs[1][0].double().numpy(), outs[1][1].double().numpy()
+    hq_g = outs[1][2].view(P + T, I).numpy()
+    off_s = (((P + T) * I + 255) // 256) * 256
+    hs_g = ws[off_s:off_s + (P + T) * (I // 128) * 4].view(torch.float32).view(P + T, I // 128).cpu().double().numpy()
+    for i in range(N_r + 1):
+        rows_i = sorted_token[offsets[i]:offsets[i + 1]] if i < N_r else np.arange(T)
+        if rows_i.size == 0:
+            continue
+        h0 = offsets[i] if i < N_r else P           # the group's first row in H
+        n = rows_i.size
+        p = O.expert_ffn_parts(xq[rows_i], xs[rows_i], experts[i])
+        da = accumulation_bound(xq[rows_i], xs[rows_i], experts[i], p["G"], p["U"])
+        flip, _ = near_tie_rows(hq_g[h0:h0 + n], hs_g[h0:h0 + n], p["a32"], da, p["hq"], p["hs"],
+                                f"expert {i} intermediate")
+        ref = p["y"]
+        if flip.size:
+            ref = ref.copy()
+            ref[flip] = O.expert_down(hq_g[h0 + flip], hs_g[h0 + flip], experts[i])
+        got = yp[offsets[i]:offsets[i + 1]] if i < N_r else ysh
+        assert_close(got, ref, f"expert {i}")
+
+
 # ---------------------------------------------------------------- failure path
 
 def test_wait_timeout_sets_error_word(lib):

@@ -36,9 +36,9 @@ def _threads():
     return max(2, min(32, os.cpu_count() or 8))
 
 
-def _build(cfg, weights_on="cuda"):
+def _build(cfg, weights_on="cuda", gather=None):
     from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
-    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I)
+    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, gather=gather)
     for slot in range(cfg.N_r + 1):
         w = workloads.expert_weights(cfg, slot, device=weights_on)
         layer.load_expert(slot, *[x.cuda() for x in w])
@@ -194,6 +194,24 @@ def test_layer_full_size(lib, name, T):
     if T is not None:
         cfg = cfg.with_tokens(T)
     _run(cfg, weights_on="cuda")
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_layer_gather_fused_equals_materialised(lib, name):
+    """The layer with the row gather fused into the GEMM and with xq_perm
+    materialised by moe_permute give the same h', bit for bit."""
+    cfg = workloads.CONFIGS[name]
+    u = workloads.activations(cfg, device="cuda")
+    e = workloads.centroids(cfg, device="cuda")
+    b = workloads.bias(cfg, device="cuda")
+    outs = []
+    for gather in (True, False):
+        layer = _build(cfg, "cuda", gather=gather)
+        bb = b.clone()
+        outs.append((layer.forward(u, e, bb).clone(), layer.y_perm.clone(), bb))
+        torch.cuda.synchronize()
+    for a_, b_ in zip(*outs):
+        assert torch.equal(a_, b_)
 
 
 def test_layer_pipelined_host_path_matches_plain():
