@@ -36,6 +36,11 @@ SIGNATURES = {
                                   _i, _i, _p, _p, _p, _z, _p]),
     "moe_grouped_gemm_fp8_gather": (_i, [_p, _p, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p,
                                          _i, _i, _p, _p, _p, _z, _p]),
+    "moe_grouped_gemm_fp8_rows_workspace": (_z, [_i, _i, _i, _i]),
+    "moe_grouped_gemm_fp8_rows": (_i, [_p, _p, _p, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p,
+                                       _i, _i, _p, _p, _p, _z, _p]),
+    "moe_group_of_rows": (_i, [_p, _i, _i, _i, _p, _p]),
+    "moe_gather_rows": (_i, [_p, _i, _p, _i, _i, _p, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _p, _i, _i, _i, _f, _p, _p]),
     "moe_debug_wait_timeout": (_i, [_i, _p]),

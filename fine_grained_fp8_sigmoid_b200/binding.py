@@ -194,6 +194,61 @@ def moe_grouped_gemm_fp8_gather(sorted_token, offsets, xq, xs, w_gate, w_up, w_d
         workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_grouped_gemm_fp8_rows_workspace(P, T, d, I):
+    return int(_lib.load().moe_grouped_gemm_fp8_rows_workspace(P, T, d, I))
+
+
+def moe_grouped_gemm_fp8_rows(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down,
+                              s_gate, s_up, s_down, y_perm, y_shared, workspace, stream=None):
+    """The grouped GEMM on P = xq_perm.shape[0] routed rows in N_groups groups
+    (weights stacked over N_groups + 1 slots, the shared expert last)."""
+    T, d = xq.shape
+    P = xq_perm.shape[0]
+    G, I, _ = w_gate.shape
+    N = G - 1
+    _want(xq_perm, torch.uint8, (P, d), "xq_perm")
+    _want(xs_perm, torch.float32, (P, d // 128), "xs_perm")
+    _want(offsets, torch.int32, (N + 1,), "offsets")
+    _want(xq, torch.uint8, (T, d), "xq")
+    _want(xs, torch.float32, (T, d // 128), "xs")
+    _want(w_gate, torch.uint8, (G, I, d), "w_gate")
+    _want(w_up, torch.uint8, (G, I, d), "w_up")
+    _want(w_down, torch.uint8, (G, d, I), "w_down")
+    _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
+    _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
+    _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
+    _want(y_perm, torch.float32, (P, d), "y_perm")
+    _want(y_shared, torch.float32, (T, d), "y_shared")
+    check("moe_grouped_gemm_fp8_rows", _lib.load().moe_grouped_gemm_fp8_rows(
+        _ptr(xq_perm), _ptr(xs_perm), _ptr(offsets), N, P, _ptr(xq), _ptr(xs), T,
+        _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(s_gate), _ptr(s_up), _ptr(s_down),
+        d, I, _ptr(y_perm), _ptr(y_shared), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_group_of_rows(offsets, modulo, out, stream=None):
+    n_groups = offsets.shape[0] - 1
+    _want(offsets, torch.int32, (n_groups + 1,), "offsets")
+    n_rows = out.shape[0]
+    _want(out, torch.int32, (n_rows,), "out")
+    check("moe_group_of_rows", _lib.load().moe_group_of_rows(
+        _ptr(offsets), n_groups, modulo, n_rows, _ptr(out), _stream(stream)))
+
+
+def moe_gather_rows(src, idx, dst, stream=None):
+    """dst[i] = src[idx[i]] along the first dimension (rows of any dtype)."""
+    n = idx.shape[0]
+    _want(idx, torch.int32, (n,), "idx")
+    if src.dtype != dst.dtype or src.shape[1:] != dst.shape[1:] or dst.shape[0] != n:
+        raise ValueError("src and dst must share dtype and row shape; dst has len(idx) rows")
+    for t, name in ((src, "src"), (dst, "dst")):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    row_bytes = dst[0].numel() * dst.element_size() if n else src[0].numel() * src.element_size()
+    check("moe_gather_rows", _lib.load().moe_gather_rows(
+        _ptr(src), src.shape[0], _ptr(idx), n, row_bytes, _ptr(dst), _stream(stream)))
+
+
 def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
     T, d = u.shape
     K_r = inv.shape[1]

@@ -854,11 +854,18 @@ static size_t counters_offset(size_t rows, int I) {
   return moe::gg::align256(moe::gg::align256(rows * I) + rows * (I / 128) * sizeof(float));
 }
 
-extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
+extern "C" size_t moe_grouped_gemm_fp8_rows_workspace(int P, int T, int d, int I) {
   (void)d;
-  if (T <= 0 || K_r <= 0 || I <= 0) return 0;
-  const size_t rows = static_cast<size_t>(T) * K_r + T;
+  if (T <= 0 || P < 0 || I <= 0) return 0;
+  const size_t rows = static_cast<size_t>(P) + T;
   return counters_offset(rows, I) + 2 * sizeof(int);
+}
+
+extern "C" size_t moe_grouped_gemm_fp8_workspace(int T, int K_r, int d, int I) {
+  if (T <= 0 || K_r <= 0 || I <= 0) return 0;
+  const long long P = static_cast<long long>(T) * K_r;
+  if (P > (1LL << 31) - 1) return 0;
+  return moe_grouped_gemm_fp8_rows_workspace(static_cast<int>(P), T, d, I);
 }
 
 // narrow tiles need the tile's [kb][token] activation-scale table to fit
@@ -875,21 +882,20 @@ extern "C" int moe_grouped_gemm_fp8_launches(int d, int I) {
 // Both entry points: the routed rows come from xq_perm/xs_perm, or (sorted_token
 // non-null) straight from xq/xs at the tokens sorted_token lists.
 static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int32_t* sorted_token,
-                        const int32_t* offsets, int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
+                        const int32_t* offsets, int N_r, long long P, const uint8_t* xq, const float* xs, int T,
                         const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down, const float* s_gate,
                         const float* s_up, const float* s_down, int d, int I, float* y_perm, float* y_shared,
                         void* workspace, size_t ws_bytes, void* stream) {
   using namespace moe;
   using namespace moe::gg;
-  MOE_CHECK_ARG(N_r >= 1 && K_r >= 1 && T >= 0 && d > 0 && I > 0);
+  MOE_CHECK_ARG(N_r >= 1 && P >= 0 && T >= 0 && d > 0 && I > 0);
   MOE_CHECK_SUPPORTED(N_r + 1 <= MAX_GROUPS && d % 256 == 0 && I % 128 == 0);
-  const long long P = static_cast<long long>(T) * K_r;
   MOE_CHECK_SUPPORTED(P + T < (1LL << 31) && static_cast<long long>(N_r + 1) * (d > I ? d : I) < (1LL << 31));
-  if (T == 0) return MOE_OK;
+  if (T == 0) return MOE_OK;   // the shared expert's rows define the call (T = 0: nothing to do)
   const bool gather = sorted_token != nullptr;
   MOE_CHECK_ARG((gather || (xq_perm && xs_perm)) && offsets && xq && xs && w_gate && w_up && w_down && s_gate &&
                 s_up && s_down && y_perm && y_shared && workspace);
-  MOE_CHECK_ARG(ws_bytes >= moe_grouped_gemm_fp8_workspace(T, K_r, d, I));
+  MOE_CHECK_ARG(ws_bytes >= moe_grouped_gemm_fp8_rows_workspace(static_cast<int>(P), T, d, I));
   MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(workspace) % 256 == 0 && reinterpret_cast<uintptr_t>(y_perm) % 16 == 0 &&
                 reinterpret_cast<uintptr_t>(y_shared) % 16 == 0);
   DeviceInfo di;
@@ -907,6 +913,9 @@ static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int3
     // one-row boxes of xq for the four-row gathers; tmA is then unused
     if (int st = make_tmap_2d(&tmXg, xq, U8, 1, T, d, 1, BK)) return st;
     tmA = tmX;
+  } else if (P == 0) {   // no routed rows: no tile reads tmA
+    tmA = tmX;
+    tmXg = tmX;
   } else {
     if (int st = make_tmap_2d(&tmA, xq_perm, U8, 1, P, d, BM, BK)) return st;
     tmXg = tmX;
@@ -915,8 +924,12 @@ static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int3
   if (int st = make_tmap_2d(&tmWu, w_up, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
   if (int st = make_tmap_2d(&tmH, H, U8, 1, rowsH, I, BM, BK)) return st;
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
-  if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
   if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
+  if (P > 0) {
+    if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
+  } else {
+    tmY = tmYs;
+  }
   // Narrow tiles only when the average routed group has at most 64 rows
   // (decode-like batches). With larger groups the few small ones gain little
   // (an N <= 64 MMA costs about as much as an N = 256 one) and their slower
@@ -977,7 +990,19 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
                                     const float* s_gate, const float* s_up, const float* s_down, int d,
                                     int I, float* y_perm, float* y_shared, void* workspace,
                                     size_t ws_bytes, void* stream) {
-  return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_r, K_r, xq, xs, T, w_gate, w_up, w_down, s_gate, s_up,
+  if (K_r < 1) return MOE_ERR_INVALID_ARG;
+  return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_r, static_cast<long long>(T) * K_r, xq, xs, T, w_gate,
+                      w_up, w_down, s_gate, s_up, s_down, d, I, y_perm, y_shared, workspace, ws_bytes, stream);
+}
+
+extern "C" int moe_grouped_gemm_fp8_rows(const uint8_t* xq_perm, const float* xs_perm, const int32_t* offsets,
+                                         int N_groups, int P, const uint8_t* xq, const float* xs, int T,
+                                         const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
+                                         const float* s_gate, const float* s_up, const float* s_down, int d, int I,
+                                         float* y_perm, float* y_shared, void* workspace, size_t ws_bytes,
+                                         void* stream) {
+  if (P < 0) return MOE_ERR_INVALID_ARG;
+  return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_groups, P, xq, xs, T, w_gate, w_up, w_down, s_gate, s_up,
                       s_down, d, I, y_perm, y_shared, workspace, ws_bytes, stream);
 }
 
@@ -987,6 +1012,8 @@ extern "C" int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token, const in
                                            const float* s_up, const float* s_down, int d, int I, float* y_perm,
                                            float* y_shared, void* workspace, size_t ws_bytes, void* stream) {
   // a null sorted_token falls to the materialised-rows check (INVALID_ARG)
-  return grouped_gemm(nullptr, nullptr, sorted_token, offsets, N_r, K_r, xq, xs, T, w_gate, w_up, w_down, s_gate,
-                      s_up, s_down, d, I, y_perm, y_shared, workspace, ws_bytes, stream);
+  if (K_r < 1) return MOE_ERR_INVALID_ARG;
+  return grouped_gemm(nullptr, nullptr, sorted_token, offsets, N_r, static_cast<long long>(T) * K_r, xq, xs, T,
+                      w_gate, w_up, w_down, s_gate, s_up, s_down, d, I, y_perm, y_shared, workspace, ws_bytes,
+                      stream);
 }

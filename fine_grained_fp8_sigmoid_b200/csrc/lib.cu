@@ -6,3 +6,4 @@
 #include "permute_noalloc.cu"
 #include "gemm.cu"
 #include "combine.cu"
+#include "ep.cu"

@@ -1,0 +1,185 @@
+"""Expert parallelism across the GPUs of one node: the DeepSeekMoE FP8 layer
+with its routed experts sharded over G ranks ("[논문 리뷰] DeepSeek-V3
+Technical Report" review, "학습 인프라 & 최적화": the model trains with EP64;
+"DeepSeek-V3 Teknik Raporu", "Problem ve motivasyon" item 2: the all-to-all
+exchange behind it is a bottleneck).
+
+Rank r holds experts [r*E, (r+1)*E), E = N_r / G, plus the shared expert
+(replicated, like the router centroids and the bias), and routes its own batch
+of T tokens. One step:
+
+  1. route, quantise (1x128) and permute the local tokens: the rows come out
+     grouped by global expert, which is grouped by owning rank;
+  2. exchange the per-expert counts (all-to-all of G x E int32), then the FP8
+     rows and their scales (all-to-all with those splits): remote rows land in
+     this GPU's memory before any kernel reads them;
+  3. group the received rows by local expert (moe_group_of_rows, then
+     moe_permute with one choice per row) and run the grouped FP8 GEMM on them
+     (moe_grouped_gemm_fp8_rows), with the shared expert on the local tokens;
+  4. put the outputs back in arrival order (moe_gather_rows) and return them
+     (all-to-all with the reverse splits): they arrive in the local
+     permutation's order, where moe_combine reads them;
+  5. the bias update uses the global load: counts summed over the ranks
+     (all-reduce), T = G * T tokens.
+
+The exchanges run through torch.distributed (NCCL on the GPUs, gloo in the
+CPU tests); every other step is an `ops` call: `GpuOps` runs the library's
+kernels, and the tests pass a CPU stand-in built on the oracle. No TMA or
+library kernel ever reads another GPU's memory.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from . import binding as B
+
+
+class GpuOps:
+    """The local steps on this GPU, through the C ABI (buffers from torch)."""
+
+    def __init__(self, d: int, I: int, E: int, device):
+        self.d, self.I, self.E = d, I, E
+        self.device = torch.device(device)
+        dev = dict(device=self.device)
+        G = E + 1                          # local experts, then the shared one
+        self.w_gate = torch.empty(G, I, d, dtype=torch.uint8, **dev)
+        self.w_up = torch.empty(G, I, d, dtype=torch.uint8, **dev)
+        self.w_down = torch.empty(G, d, I, dtype=torch.uint8, **dev)
+        self.s_gate = torch.empty(G, I // 128, d // 128, dtype=torch.float32, **dev)
+        self.s_up = torch.empty(G, I // 128, d // 128, dtype=torch.float32, **dev)
+        self.s_down = torch.empty(G, d // 128, I // 128, dtype=torch.float32, **dev)
+
+    def load_expert(self, local_slot, w_gate, w_up, w_down):
+        B.moe_quant_128x128(w_gate, self.w_gate[local_slot], self.s_gate[local_slot])
+        B.moe_quant_128x128(w_up, self.w_up[local_slot], self.s_up[local_slot])
+        B.moe_quant_128x128(w_down, self.w_down[local_slot], self.s_down[local_slot])
+
+    def _empty(self, *shape, dtype):
+        return torch.empty(*shape, dtype=dtype, device=self.device)
+
+    def route(self, u, e, b, K):
+        T = u.shape[0]
+        idx, gates = self._empty(T, K, dtype=torch.int32), self._empty(T, K, dtype=torch.float32)
+        B.moe_route(u, e, b, K, idx, gates)
+        return idx, gates
+
+    def quant(self, u):
+        T, d = u.shape
+        xq, xs = self._empty(T, d, dtype=torch.uint8), self._empty(T, d // 128, dtype=torch.float32)
+        B.moe_quant_1x128(u, xq, xs)
+        return xq, xs
+
+    def permute(self, idx, N, xq, xs):
+        T, K = idx.shape
+        d = xq.shape[1]
+        counts, offsets = self._empty(N, dtype=torch.int32), self._empty(N + 1, dtype=torch.int32)
+        st, inv = self._empty(T * K, dtype=torch.int32), self._empty(T, K, dtype=torch.int32)
+        xqp, xsp = self._empty(T * K, d, dtype=torch.uint8), self._empty(T * K, d // 128, dtype=torch.float32)
+        ws = self._empty(max(B.moe_permute_workspace(T, N), 16), dtype=torch.uint8)
+        B.moe_permute(idx, N, counts, offsets, st, inv, ws, xq, xs, xqp, xsp)
+        return counts, offsets, inv, xqp, xsp
+
+    def group_of_rows(self, offsets, modulo, n_rows):
+        out = self._empty(n_rows, dtype=torch.int32)
+        B.moe_group_of_rows(offsets, modulo, out)
+        return out
+
+    def experts(self, xq_perm, xs_perm, offsets, xq, xs):
+        P, T = xq_perm.shape[0], xq.shape[0]
+        y_perm, y_sh = self._empty(P, self.d, dtype=torch.float32), self._empty(T, self.d, dtype=torch.float32)
+        ws = self._empty(max(B.moe_grouped_gemm_fp8_rows_workspace(P, T, self.d, self.I), 256), dtype=torch.uint8)
+        B.moe_grouped_gemm_fp8_rows(xq_perm, xs_perm, offsets, xq, xs, self.w_gate, self.w_up, self.w_down,
+                                    self.s_gate, self.s_up, self.s_down, y_perm, y_sh, ws)
+        return y_perm, y_sh
+
+    def gather_rows(self, src, idx):
+        dst = self._empty(idx.shape[0], *src.shape[1:], dtype=src.dtype)
+        B.moe_gather_rows(src, idx, dst)
+        return dst
+
+    def combine(self, u, y_perm, y_shared, inv, gates):
+        out = torch.empty_like(u)
+        B.moe_combine(u, y_perm, y_shared, inv, gates, out)
+        return out
+
+    def bias_update(self, b, counts, T, K, gamma=0.001):
+        mom = self._empty(1, dtype=torch.float32)
+        B.moe_bias_update(b, counts, T, K, gamma, mom)
+        return mom
+
+
+def split_plan(counts_local: np.ndarray, recv_counts: np.ndarray, G: int, E: int):
+    """Host-side plan of one exchange from the per-expert counts.
+
+    counts_local [G*E]: rows this rank sends to each global expert, grouped by
+    owning rank. recv_counts [G, E]: rows each source rank sends to each of
+    this rank's experts. Returns (send_splits [G], recv_splits [G], recv
+    offsets over the G*E (source, expert) groups of the received rows)."""
+    send = counts_local.reshape(G, E).sum(axis=1)
+    recv = recv_counts.sum(axis=1)
+    off = np.concatenate([[0], np.cumsum(recv_counts.reshape(-1))]).astype(np.int32)
+    return send.astype(np.int64).tolist(), recv.astype(np.int64).tolist(), off
+
+
+class ExpertParallelMoE:
+    """The layer on this rank's T tokens, routed experts sharded over the
+    ranks of `group`. load_expert takes the global expert index (slot N_r is
+    the shared expert); ranks ignore the experts they do not own."""
+
+    def __init__(self, T, d, N_r, K_r, I, group=None, ops=None, device="cuda"):
+        self.group = group
+        self.G = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if N_r % self.G:
+            raise ValueError("N_r must be a multiple of the number of ranks")
+        self.T, self.d, self.N_r, self.K_r, self.I = T, d, N_r, K_r, I
+        self.E = N_r // self.G
+        self.ops = ops if ops is not None else GpuOps(d, I, self.E, device)
+        self.last = {}
+
+    def owns(self, slot):
+        return slot == self.N_r or slot // self.E == self.rank
+
+    def load_expert(self, slot, w_gate, w_up, w_down):
+        if slot == self.N_r:
+            self.ops.load_expert(self.E, w_gate, w_up, w_down)
+        elif self.owns(slot):
+            self.ops.load_expert(slot - self.rank * self.E, w_gate, w_up, w_down)
+
+    def _a2a(self, out, inp, out_splits, in_splits):
+        dist.all_to_all_single(out, inp, out_splits, in_splits, group=self.group)
+        return out
+
+    def forward(self, u, e, b, update_bias=True, gamma=0.001):
+        ops, G, E, K = self.ops, self.G, self.E, self.K_r
+        T, d = u.shape
+        idx, gates = ops.route(u, e, b, K)
+        xq, xs = ops.quant(u)
+        counts, _, inv, xq_perm, xs_perm = ops.permute(idx, self.N_r, xq, xs)
+
+        # counts first: rows per (this rank -> expert of rank j) to each j
+        recv_counts = self._a2a(torch.empty_like(counts), counts, [E] * G, [E] * G)
+        send, recv, roff = split_plan(counts.cpu().numpy(), recv_counts.cpu().numpy().reshape(G, E), G, E)
+        R = int(sum(recv))
+        rxq = self._a2a(xq_perm.new_empty(R, d), xq_perm, recv, send)
+        rxs = self._a2a(xs_perm.new_empty(R, d // 128), xs_perm, recv, send)
+
+        # received rows are grouped by (source, local expert): regroup by expert
+        roff_d = torch.from_numpy(roff).to(counts.device)
+        local_e = ops.group_of_rows(roff_d, E, R)
+        lcounts, loff, linv, lxq, lxs = ops.permute(local_e.view(R, 1), E, rxq, rxs)
+        y_loc, y_sh = ops.experts(lxq, lxs, loff, xq, xs)
+        y_back = ops.gather_rows(y_loc, linv.view(R))          # arrival order
+        y_perm = self._a2a(y_loc.new_empty(T * K, d), y_back, send, recv)
+
+        out = ops.combine(u, y_perm, y_sh, inv, gates)
+        mom = None
+        if update_bias:
+            total = counts.clone()
+            dist.all_reduce(total, op=dist.ReduceOp.SUM, group=self.group)
+            mom = ops.bias_update(b, total, G * T, K, gamma)
+        self.last = dict(topk_idx=idx, gates=gates, counts=counts, recv_counts=recv_counts, send=send,
+                         recv=recv, local_counts=lcounts, y_perm=y_perm, y_shared=y_sh, max_over_mean=mom)
+        return out

@@ -259,6 +259,50 @@ MOE_API int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_grouped_gemm_fp8_rows_workspace / moe_grouped_gemm_fp8_rows: the grouped
+ * GEMM with an explicit count P of routed rows in N_groups groups instead of
+ * P = T * K_r; the shared expert runs on T rows of xq (slot N_groups). Used
+ * where the routed rows are not this batch's T * K_r pairs: under expert
+ * parallelism a GPU runs its local experts on the rows the other GPUs sent
+ * it ("[논문 리뷰] DeepSeek-V3 Technical Report" review, "학습 인프라 &
+ * 최적화": EP64). Same products, scales, layouts and limits as
+ * moe_grouped_gemm_fp8 (weights stacked over N_groups + 1 slots); P may be 0
+ * (then xq_perm, xs_perm and y_perm may be NULL); T must be >= 1.
+ */
+MOE_API size_t moe_grouped_gemm_fp8_rows_workspace(int P, int T, int d, int I);
+MOE_API int moe_grouped_gemm_fp8_rows(const uint8_t* xq_perm, const float* xs_perm,
+                         const int32_t* offsets, int N_groups, int P,
+                         const uint8_t* xq, const float* xs, int T,
+                         const uint8_t* w_gate, const uint8_t* w_up,
+                         const uint8_t* w_down, const float* s_gate,
+                         const float* s_up, const float* s_down, int d, int I,
+                         float* y_perm, float* y_shared,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_group_of_rows: out[p] = g mod modulo for every row p of a grouped layout
+ * (offsets[g] <= p < offsets[g+1], offsets [n_groups+1] int32 on the device,
+ * n_rows = offsets[n_groups]). Under expert parallelism the rows a GPU
+ * receives are grouped by (source GPU, local expert): with modulo = local
+ * experts this yields each row's local expert. No counterpart on the pages
+ * (row bookkeeping around the all-to-all they describe, "DeepSeek-V3 Teknik
+ * Raporu", "Problem ve motivasyon" item 2).
+ */
+MOE_API int moe_group_of_rows(const int32_t* offsets, int n_groups, int modulo,
+                      int n_rows, int32_t* out, void* stream);
+
+/*
+ * moe_gather_rows: dst row i = src row idx[i] for i < n; rows of row_bytes
+ * bytes (a multiple of 16), src holds n_src rows; src and dst 16-byte
+ * aligned. An index outside [0, n_src) is skipped and recorded as
+ * MOE_ERR_INVALID_ARG in the device error word. Puts expert outputs back into
+ * the order the rows arrived in before they return to their GPUs. No
+ * counterpart on the pages.
+ */
+MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* idx, int n,
+                    int row_bytes, void* dst, void* stream);
+
+/*
  * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
  * ("DeepSeek-V3 Teknik Raporu", Yöntem 2, the h'_t equation). The sum is FP32
  * in the fixed order u, shared, k = 0..K_r-1.
