@@ -700,13 +700,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      // The row's activation scale (a different cache line for every
+      // thread) is loaded two K blocks ahead, the weight block's scales (one
+      // line for the whole CTA) one block ahead.
       float sa_n = valid ? __ldg(sa_ptr) : 0.0f;
+      float sa_n2 = (valid && KB > 1) ? __ldg(sa_ptr + 1) : 0.0f;
       float s0_n = __ldg(sb0), s1_n = __ldg(sb1);
       bool ok = true;
       for (int kb = 0; kb < KB; ++kb) {
         const float sa = sa_n, s0 = s0_n, s1 = s1_n;
-        if (kb + 1 < KB) {  // next block's scales, loaded one block ahead
-          sa_n = valid ? __ldg(sa_ptr + kb + 1) : 0.0f;
+        sa_n = sa_n2;
+        if (kb + 2 < KB) sa_n2 = valid ? __ldg(sa_ptr + kb + 2) : 0.0f;
+        if (kb + 1 < KB) {
           s0_n = __ldg(sb0 + kb + 1);
           s1_n = __ldg(sb1 + kb + 1);
         }
