@@ -206,6 +206,80 @@ def expert_ffn(xq, xs, w: dict):
 
 
 # --------------------------------------------------------------------------
+# Backward of one expert FFN in the same FP8 scheme. The pages train in FP8
+# ([TR] Temel fikirler, FP8 bullet: E4M3 on all tensors, activations in 1x128
+# tiles, weights in 128x128 blocks) and print no backward details; the
+# readings taken:
+#  * every GEMM of the backward has FP8 operands, E4M3 like the forward's;
+#  * an operand's granularity follows its role in the product: the operand
+#    whose rows are the product's rows (the "activation" role) has one scale
+#    per 1x128 tile along the contraction, the other (the "weight" role) one
+#    scale per 128x128 block; before quantisation a value is rounded to FP32;
+#  * the requantisation of the intermediate is a cast in the backward (its
+#    gradient passes through unchanged);
+#  * dgrad uses the forward's weight codes and scales (transposed exactly);
+#    wgrad contracts over the expert's tokens, zero-padded to a multiple of
+#    128, with the forward's FP8 activations (X and H as the forward used
+#    them) requantised in 128x128 blocks and the gradients in 1x128 tiles.
+# --------------------------------------------------------------------------
+
+def dsilu(x: np.ndarray) -> np.ndarray:
+    """d/dx silu(x) = sigma(x) (1 + x (1 - sigma(x)))."""
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-x))
+    return s * (1.0 + x * (1.0 - s))
+
+
+def _fp8_act(x, quantize):
+    """An operand in the activation role: 1x128 tiles along the rows."""
+    return dequant_1x128(*quant_1x128(round_fp32(x))) if quantize else x
+
+
+def _fp8_blocks(x, quantize):
+    """An operand in the weight role: 128x128 blocks."""
+    return dequant_128x128(*quant_128x128(round_fp32(x))) if quantize else x
+
+
+def _pad_rows(x, m):
+    return np.concatenate([x, np.zeros((m - x.shape[0],) + x.shape[1:])]) if m > x.shape[0] else x
+
+
+def expert_ffn_backward(xq, xs, w: dict, dy, quantize: bool = True) -> dict:
+    """Gradients of Y = H W_down^T, H = q(silu(X W_gate^T) * (X W_up^T)) for
+    one expert's FP8 rows (xq, xs) given dY [m, d].
+
+    Returns dict with dx [m, d], dw_gate [I, d], dw_up [I, d], dw_down [d, I]
+    and the intermediates (G, U, dh, dg, du). quantize=False drops every
+    backward quantisation (the forward's FP8 operands stay): then the result
+    is the plain float64 derivative of the forward as executed.
+    """
+    X = dequant_1x128(xq, xs)
+    Wg = dequant_128x128(w["gate_q"], w["gate_s"])
+    Wu = dequant_128x128(w["up_q"], w["up_s"])
+    Wd = dequant_128x128(w["down_q"], w["down_s"])
+    G, U = X @ Wg.T, X @ Wu.T
+    a32 = round_fp32(silu(G) * U)
+    H = dequant_1x128(*quant_1x128(a32))
+    m = X.shape[0]
+    # dgrad: dH = dY W_down, then through SwiGLU, dX = dG W_gate + dU W_up
+    dh = _fp8_act(np.asarray(dy, np.float64), quantize) @ Wd
+    dg = dh * U * dsilu(G)
+    du = dh * silu(G)
+    dgu = _fp8_act(np.concatenate([dg, du], axis=1), quantize)
+    I = dg.shape[1]
+    dx = dgu[:, :I] @ Wg + dgu[:, I:] @ Wu
+    # wgrad: contractions over the tokens, padded to a multiple of 128
+    mp = -(-m // 128) * 128
+    t_act = lambda g: _fp8_act(_pad_rows(g, mp).T, quantize)     # [features, tokens]
+    t_blk = lambda v: _fp8_blocks(_pad_rows(v, mp).T, quantize)
+    dw_down = t_act(dy) @ t_blk(H).T
+    Xt = t_blk(X)
+    dw_gate = t_act(dg) @ Xt.T
+    dw_up = t_act(du) @ Xt.T
+    return dict(dx=dx, dw_gate=dw_gate, dw_up=dw_up, dw_down=dw_down, G=G, U=U, dh=dh, dg=dg, du=du, H=H)
+
+
+# --------------------------------------------------------------------------
 # Combine ([TR] Yöntem 2, h'_t = u_t + sum_s FFN^(s)(u_t) + sum_i g_{i,t} FFN^(r)_i(u_t))
 # --------------------------------------------------------------------------
 

@@ -393,3 +393,74 @@ def test_tiny_forward_is_finite_and_near_residual_scale():
     assert r["out"].shape == (cfg.T, cfg.d)
     # the expert contribution is small next to the N(0,1) residual
     assert np.abs(r["out"] - u).max() < 1.0
+
+
+# ---------------------------------------------------------------- backward
+
+def test_dsilu_against_autograd():
+    x = np.linspace(-30, 30, 601)
+    t = torch.tensor(x, dtype=torch.float64, requires_grad=True)
+    torch.nn.functional.silu(t).sum().backward()
+    assert np.allclose(moe.dsilu(x), t.grad.numpy(), rtol=1e-13, atol=1e-15)
+    assert moe.dsilu(np.array([0.0]))[0] == 0.5
+
+
+def _bwd_case(m=37, d=256, I=128, seed=3):
+    rng = np.random.default_rng(seed)
+    xq, xs = moe.quant_1x128(rng.standard_normal((m, d)))
+    w = moe.quantise_expert(rng.standard_normal((I, d)) * 0.05, rng.standard_normal((I, d)) * 0.05,
+                            rng.standard_normal((d, I)) * 0.05)
+    dy = round_bf16(rng.standard_normal((m, d)))
+    return xq, xs, w, dy
+
+
+def test_expert_backward_without_quantisation_is_the_autograd_derivative():
+    # the wiring (transposes, operand roles, the SwiGLU derivative, the
+    # requantisation passed through) against torch float64 autograd of the
+    # forward as executed: the same dequantised operands, H = a + (q(a) - a)
+    xq, xs, w, dy = _bwd_case()
+    r = moe.expert_ffn_backward(xq, xs, w, dy, quantize=False)
+    T = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)
+    X = T(moe.dequant_1x128(xq, xs))
+    Wg, Wu, Wd = (T(moe.dequant_128x128(w[k + "_q"], w[k + "_s"])) for k in ("gate", "up", "down"))
+    a = torch.nn.functional.silu(X @ Wg.T) * (X @ Wu.T)
+    hq, hs = moe.quant_1x128(round_fp32(a.detach().numpy()))
+    H = a + torch.tensor(moe.dequant_1x128(hq, hs) - a.detach().numpy())   # the cast, as a constant shift
+    Y = H @ Wd.T
+    Y.backward(torch.tensor(dy))
+    for got, t in [(r["dx"], X), (r["dw_gate"], Wg), (r["dw_up"], Wu), (r["dw_down"], Wd)]:
+        assert np.allclose(got, t.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_expert_backward_quantised_operands_stay_within_the_fp8_error():
+    # with the backward's own FP8 quantisations the gradients move by about
+    # the E4M3 step (2^-4 relative per operand), not more
+    xq, xs, w, dy = _bwd_case(m=300, d=512, I=256, seed=5)
+    q = moe.expert_ffn_backward(xq, xs, w, dy)
+    e = moe.expert_ffn_backward(xq, xs, w, dy, quantize=False)
+    for k in ("dx", "dw_gate", "dw_up", "dw_down"):
+        rel = np.linalg.norm(q[k] - e[k]) / np.linalg.norm(e[k])
+        assert 1e-4 < rel < 0.08, (k, rel)
+
+
+def test_expert_backward_exact_on_representable_values():
+    # one token row: x = 1, weights 2^-7 everywhere, d = I = 128: G = U = 1,
+    # a = silu(1); dY = 1 everywhere (one value per tile: code 448, scale
+    # fl32(1/448)). dH = 128 * 2^-7 * q(1); dG = dH U dsilu(1), dU = dH silu(1) (each tile one
+    # value, so its code is +-448 and the quantisation exact up to the FP32
+    # rounding of the scale); dX = 128 * 2^-7 * (dG + dU)
+    d = I = 128
+    xq = np.full((1, d), 0x38, np.uint8)
+    w = dict(gate_q=np.full((I, d), 0x04, np.uint8), gate_s=np.ones((1, 1)),
+             up_q=np.full((I, d), 0x04, np.uint8), up_s=np.ones((1, 1)),
+             down_q=np.full((d, I), 0x04, np.uint8), down_s=np.ones((1, 1)))
+    r = moe.expert_ffn_backward(xq, np.ones((1, 1)), w, np.ones((1, d)))
+    sig = 1 / (1 + math.exp(-1.0))
+    q = lambda v: 448.0 * float(np.float32(float(np.float32(v)) / 448.0))   # a tile of one value
+    dh = q(1.0)                                  # dY = 1 dequantises to 448 * fl32(1/448)
+    dg, du = q(dh * sig * (1 + (1 - sig))), q(dh * sig)
+    assert np.all(r["dh"] == dh)
+    assert np.allclose(r["dx"], dg + du, rtol=0, atol=1e-15)
+    # wgrad: one token (padded to 128 with zeros): dW_down[j][i] = dY * H
+    h = q(float(np.float32(sig)))
+    assert np.allclose(r["dw_down"], h, rtol=2 ** -10)
