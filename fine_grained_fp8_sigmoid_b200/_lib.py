@@ -41,6 +41,12 @@ SIGNATURES = {
                                        _i, _i, _p, _p, _p, _z, _p]),
     "moe_group_of_rows": (_i, [_p, _i, _i, _i, _p, _p]),
     "moe_gather_rows": (_i, [_p, _i, _p, _i, _i, _p, _p]),
+    "moe_grouped_scaled_gemm_fp8_workspace": (_z, []),
+    "moe_grouped_scaled_gemm_fp8": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _i, _i, _p, _p, _z, _p]),
+    "moe_swiglu_backward_quant": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p]),
+    "moe_quant_1x128_t": (_i, [_p, _i, _i, _i, _p, _p, _i, _i, _p, _p, _p]),
+    "moe_quant_128x128_t": (_i, [_p, _p, _i, _i, _p, _p, _i, _i, _p, _p, _p]),
+    "moe_transpose": (_i, [_p, _i, _i, _i, _i, _p, _i, _i, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _p, _i, _i, _i, _f, _p, _p]),
     "moe_debug_wait_timeout": (_i, [_i, _p]),

@@ -249,6 +249,93 @@ def moe_gather_rows(src, idx, dst, stream=None):
         _ptr(src), src.shape[0], _ptr(idx), n, row_bytes, _ptr(dst), _stream(stream)))
 
 
+def moe_grouped_scaled_gemm_fp8_workspace():
+    return int(_lib.load().moe_grouped_scaled_gemm_fp8_workspace())
+
+
+def moe_grouped_scaled_gemm_fp8(a, a_s, offsets, P, b, b_s, c, workspace, stream=None):
+    """c = a b_g^T: a [P+T][K] (1x128 scales a_s), b [N_groups+1][N][K] (128x128
+    scales b_s); rows of group g use slot g, the last T rows the last slot."""
+    R, K = a.shape
+    G, N, _ = b.shape
+    T = R - P
+    _want(a, torch.uint8, (R, K), "a")
+    _want(a_s, torch.float32, (R, K // 128), "a_s")
+    _want(offsets, torch.int32, (G,), "offsets")
+    _want(b, torch.uint8, (G, N, K), "b")
+    _want(b_s, torch.float32, (G, N // 128, K // 128), "b_s")
+    _want(c, torch.float32, (R, N), "c")
+    check("moe_grouped_scaled_gemm_fp8", _lib.load().moe_grouped_scaled_gemm_fp8(
+        _ptr(a), _ptr(a_s), _ptr(offsets), G - 1, P, T, _ptr(b), _ptr(b_s), K, N, _ptr(c),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def moe_swiglu_backward_quant(g, u, dh, dgu, q, qs, stream=None):
+    R, I = g.shape
+    for t, n in ((g, "g"), (u, "u"), (dh, "dh")):
+        _want(t, torch.float32, (R, I), n)
+    _opt(dgu, torch.float32, (R, 2 * I), "dgu")
+    _want(q, torch.uint8, (R, 2 * I), "q")
+    _want(qs, torch.float32, (R, 2 * I // 128), "qs")
+    check("moe_swiglu_backward_quant", _lib.load().moe_swiglu_backward_quant(
+        _ptr(g), _ptr(u), _ptr(dh), R, I, _ptr(dgu), _ptr(q), _ptr(qs), _stream(stream)))
+
+
+def _ld(x):
+    if not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a CUDA matrix with unit column stride")
+    return x.stride(0)
+
+
+def moe_quant_1x128_t(x, src_off, dst_off, q, s, stream=None):
+    """x [rows][cols] FP32 or BF16 (a column slice of a wider row-major tensor
+    is allowed) -> per group g a [cols][K_g] block of q (flat, cols * Ktot
+    bytes) and a [cols][K_g/128] block of s (flat)."""
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("x must be FP32 or BF16")
+    cols = x.shape[1]
+    Ktot = q.numel() // cols
+    n = src_off.shape[0] - 1
+    _want(src_off, torch.int32, (n + 1,), "src_off")
+    _want(dst_off, torch.int32, (n + 1,), "dst_off")
+    _want(q, torch.uint8, (cols * Ktot,), "q")
+    _want(s, torch.float32, (cols * Ktot // 128,), "s")
+    check("moe_quant_1x128_t", _lib.load().moe_quant_1x128_t(
+        _ptr(x), int(x.dtype == torch.bfloat16), _ld(x), cols, _ptr(src_off), _ptr(dst_off), n, Ktot,
+        _ptr(q), _ptr(s), _stream(stream)))
+
+
+def moe_quant_128x128_t(xq, xs, src_off, dst_off, q, s, stream=None):
+    """xq [rows][cols] E4M3 with 1x128 scales xs -> per group g a [cols][K_g]
+    block of q (flat) in 128x128 blocks, scales [cols/128][K_g/128] (flat)."""
+    rows, cols = xq.shape
+    Ktot = q.numel() // cols
+    n = src_off.shape[0] - 1
+    _want(xq, torch.uint8, (rows, cols), "xq")
+    _want(xs, torch.float32, (rows, cols // 128), "xs")
+    _want(src_off, torch.int32, (n + 1,), "src_off")
+    _want(dst_off, torch.int32, (n + 1,), "dst_off")
+    _want(q, torch.uint8, (cols * Ktot,), "q")
+    _want(s, torch.float32, ((cols // 128) * (Ktot // 128),), "s")
+    check("moe_quant_128x128_t", _lib.load().moe_quant_128x128_t(
+        _ptr(xq), _ptr(xs), cols, cols, _ptr(src_off), _ptr(dst_off), n, Ktot, _ptr(q), _ptr(s),
+        _stream(stream)))
+
+
+def moe_transpose(src, dst, dst_col=0, stream=None):
+    """dst[b][j][dst_col + i] = src[b][i][j] (uint8 or float32, 3-D, contiguous)."""
+    if src.dtype != dst.dtype or src.dtype not in (torch.uint8, torch.float32):
+        raise ValueError("src and dst: both uint8 or both float32")
+    B, rows, cols = src.shape
+    if dst.shape[0] != B or dst.shape[1] != cols or dst.shape[2] < dst_col + rows:
+        raise ValueError("dst must be [batch][cols][>= dst_col + rows]")
+    for t, n in ((src, "src"), (dst, "dst")):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CUDA tensor")
+    check("moe_transpose", _lib.load().moe_transpose(
+        _ptr(src), src.element_size(), B, rows, cols, _ptr(dst), dst.shape[2], dst_col, _stream(stream)))
+
+
 def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
     T, d = u.shape
     K_r = inv.shape[1]

@@ -7,7 +7,7 @@
 //                       layout, from its offsets: on the receiving GPU, the
 //                       local expert of each received row.
 //   moe_gather_rows   - dst[i] = src[idx[i]] for rows of any width (a
-//                       multiple of 16 bytes): expert outputs back into
+//                       multiple of 4 bytes): expert outputs back into
 //                       arrival order before they return.
 #include "host.cuh"
 
@@ -26,10 +26,11 @@ __global__ void __launch_bounds__(256) group_of_rows_kernel(const int32_t* __res
   out[p] = lo % modulo;
 }
 
-// One warp per row, 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ src, int n_src,
+// One warp per row, in vectors of V (16-byte or 4-byte words).
+template <typename V>
+__global__ void __launch_bounds__(256) gather_rows_kernel(const V* __restrict__ src, int n_src,
                                                           const int32_t* __restrict__ idx, int n, int vec_per_row,
-                                                          uint4* __restrict__ dst) {
+                                                          V* __restrict__ dst) {
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
   for (long long i = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); i < n; i += warps) {
     const int r = __ldg(idx + i);
@@ -37,8 +38,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restric
       if (lane_id() == 0) set_device_error(MOE_ERR_INVALID_ARG);
       continue;
     }
-    const uint4* s = src + static_cast<size_t>(r) * vec_per_row;
-    uint4* d = dst + static_cast<size_t>(i) * vec_per_row;
+    const V* s = src + static_cast<size_t>(r) * vec_per_row;
+    V* d = dst + static_cast<size_t>(i) * vec_per_row;
     for (int v = lane_id(); v < vec_per_row; v += 32) d[v] = __ldg(s + v);
   }
 }
@@ -63,16 +64,22 @@ extern "C" int moe_gather_rows(const void* src, int n_src, const int32_t* idx, i
                                void* stream) {
   using namespace moe;
   MOE_CHECK_ARG(n_src >= 0 && n >= 0 && row_bytes > 0);
-  MOE_CHECK_SUPPORTED(row_bytes % 16 == 0);
+  MOE_CHECK_SUPPORTED(row_bytes % 4 == 0);
   if (n == 0) return MOE_OK;
   MOE_CHECK_ARG(src && idx && dst && n_src > 0);
-  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(src) % 16 == 0 && reinterpret_cast<uintptr_t>(dst) % 16 == 0);
+  const bool wide = row_bytes % 16 == 0 && reinterpret_cast<uintptr_t>(src) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(dst) % 16 == 0;
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(src) % 4 == 0 && reinterpret_cast<uintptr_t>(dst) % 4 == 0);
   DeviceInfo di;
   if (int st = device_info(&di)) return st;
   long long blocks = (static_cast<long long>(n) + 7) / 8;
   const long long cap = static_cast<long long>(di.sm_count) * 16;
   if (blocks > cap) blocks = cap;
-  ep::gather_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
-      static_cast<const uint4*>(src), n_src, idx, n, row_bytes / 16, static_cast<uint4*>(dst));
+  if (wide)
+    ep::gather_rows_kernel<uint4><<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+        static_cast<const uint4*>(src), n_src, idx, n, row_bytes / 16, static_cast<uint4*>(dst));
+  else
+    ep::gather_rows_kernel<uint32_t><<<static_cast<unsigned>(blocks), 256, 0, as_stream(stream)>>>(
+        static_cast<const uint32_t*>(src), n_src, idx, n, row_bytes / 4, static_cast<uint32_t*>(dst));
   return launch_status("moe_gather_rows");
 }

@@ -1022,3 +1022,63 @@ extern "C" int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token, const in
                       w_gate, w_up, w_down, s_gate, s_up, s_down, d, I, y_perm, y_shared, workspace, ws_bytes,
                       stream);
 }
+
+// A grouped scaled GEMM on the down-projection kernel: C = A B_g^T with A in
+// the activation role (1x128 tiles along K) and B in the weight role (128x128
+// blocks), the same FP32 promotion per 128-wide K block. The backward's
+// products are of this form (dgrad with transposed weights; wgrad with one
+// group whose rows are features and whose K is the expert's tokens).
+extern "C" size_t moe_grouped_scaled_gemm_fp8_workspace(void) { return 256; }
+
+extern "C" int moe_grouped_scaled_gemm_fp8(const uint8_t* a, const float* a_s, const int32_t* offsets, int N_groups,
+                                           int P, int T, const uint8_t* b, const float* b_s, int K, int N, float* c,
+                                           void* workspace, size_t ws_bytes, void* stream) {
+  using namespace moe;
+  using namespace moe::gg;
+  MOE_CHECK_ARG(N_groups >= 0 && P >= 0 && T >= 1 && K > 0 && N > 0);
+  MOE_CHECK_SUPPORTED(N_groups + 1 <= MAX_GROUPS && K % BK == 0 && N % BN == 0);
+  MOE_CHECK_SUPPORTED(static_cast<long long>(P) + T < (1LL << 31) &&
+                      static_cast<long long>(N_groups + 1) * N < (1LL << 31));
+  MOE_CHECK_ARG(a && a_s && offsets && b && b_s && c && workspace);
+  MOE_CHECK_ARG(ws_bytes >= moe_grouped_scaled_gemm_fp8_workspace());
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(workspace) % 16 == 0 && reinterpret_cast<uintptr_t>(c) % 16 == 0);
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  cudaStream_t s = as_stream(stream);
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMap tmA, tmB, tmC, tmCs;
+  if (int st = make_tmap_2d(&tmA, a, U8, 1, static_cast<uint64_t>(P) + T, K, BM, BK)) return st;
+  if (int st = make_tmap_2d(&tmB, b, U8, 1, static_cast<uint64_t>(N_groups + 1) * N, K, BN, BK)) return st;
+  float* c_sh = c + static_cast<size_t>(P) * N;
+  if (int st = make_tmap_y(&tmCs, c_sh, T, N)) return st;
+  if (P > 0) {
+    if (int st = make_tmap_y(&tmC, c, P, N)) return st;
+  } else {
+    tmC = tmCs;
+  }
+  Args args{};
+  args.offsets = offsets;
+  args.N_r = N_groups;
+  args.T = T;
+  args.P = P;
+  args.d = N;          // the down kernel's output width
+  args.I = K;          // and its contraction
+  args.Hs = const_cast<float*>(a_s);
+  args.s_down = b_s;
+  args.y_perm = c;
+  args.y_shared = c_sh;
+  args.narrow_max = 0;
+  args.sorted_token = nullptr;
+  args.tile_counter = static_cast<int*>(workspace);
+  if (int st = cuda_status(cudaMemsetAsync(workspace, 0, sizeof(int), s), "scaled GEMM: tile counter")) return st;
+  const long long m_tiles = (P + BM - 1) / BM + (P < N_groups ? P : N_groups) + (T + BM - 1) / BM;
+  const long long tiles = m_tiles * (N / BN);
+  const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
+  auto k2 = grouped_gemm_kernel<2>;
+  constexpr size_t sm2 = smem_bytes<2>();
+  if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
+                           "smem attribute (scaled GEMM)"))
+    return st;
+  k2<<<grid, THREADS, sm2, s>>>(tmA, tmA, tmB, tmB, tmC, tmCs, tmA, args);
+  return launch_status("scaled GEMM launch");
+}

@@ -7,3 +7,4 @@
 #include "gemm.cu"
 #include "combine.cu"
 #include "ep.cu"
+#include "backward.cu"

@@ -293,14 +293,92 @@ MOE_API int moe_group_of_rows(const int32_t* offsets, int n_groups, int modulo,
 
 /*
  * moe_gather_rows: dst row i = src row idx[i] for i < n; rows of row_bytes
- * bytes (a multiple of 16), src holds n_src rows; src and dst 16-byte
- * aligned. An index outside [0, n_src) is skipped and recorded as
+ * bytes (a multiple of 4), src holds n_src rows; src and dst 4-byte aligned
+ * (16-byte rows and alignment move in 16-byte words). An index outside [0, n_src) is skipped and recorded as
  * MOE_ERR_INVALID_ARG in the device error word. Puts expert outputs back into
  * the order the rows arrived in before they return to their GPUs. No
  * counterpart on the pages.
  */
 MOE_API int moe_gather_rows(const void* src, int n_src, const int32_t* idx, int n,
                     int row_bytes, void* dst, void* stream);
+
+/*
+ * ---------------------------------------------------------------- backward
+ * The expert FFN's backward in the same FP8 scheme ("DeepSeek-V3 Teknik
+ * Raporu", Temel fikirler, FP8 bullet: training in FP8 with E4M3 on all
+ * tensors, activations in 1x128 tiles, weights in 128x128 blocks; the pages
+ * print no backward details). Every backward GEMM has E4M3 operands; the
+ * operand in the activation role (its rows are the product's rows) has one
+ * FP32 scale per 1x128 tile along the contraction, the other one per 128x128
+ * block; the requantisation of the intermediate is a cast (its gradient passes
+ * through). wgrad contracts over an expert's tokens, each group's tokens
+ * zero-padded to a multiple of 128.
+ */
+
+/*
+ * moe_grouped_scaled_gemm_fp8: C = A B_g^T on the grouped GEMM kernel, FP32
+ * promotion per 128-wide K block.
+ *   a, a_s     [P+T][K] E4M3 and [P+T][K/128] FP32 (1x128 tiles); rows
+ *              offsets[g]..offsets[g+1] (g < N_groups, offsets[N_groups] = P)
+ *              use B slot g, the last T rows slot N_groups
+ *   offsets    [N_groups+1] int32 (device); N_groups may be 0 (one group)
+ *   b, b_s     [N_groups+1][N][K] E4M3, [N_groups+1][N/128][K/128] FP32
+ *   c          [P+T][N] FP32 (out)
+ *   workspace  moe_grouped_scaled_gemm_fp8_workspace() bytes (a tile counter)
+ * Limits: K a multiple of 128, N a multiple of 256, T >= 1.
+ */
+MOE_API size_t moe_grouped_scaled_gemm_fp8_workspace(void);
+MOE_API int moe_grouped_scaled_gemm_fp8(const uint8_t* a, const float* a_s,
+                         const int32_t* offsets, int N_groups, int P, int T,
+                         const uint8_t* b, const float* b_s, int K, int N,
+                         float* c, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * moe_swiglu_backward_quant: for rows r < R and columns i < I,
+ *   dG = dH U silu'(G),  dU = dH silu(G),  silu'(x) = s(x)(1 + x(1 - s(x)))
+ * with s the sigmoid, then [dG | dU] ([R][2I]) quantised in 1x128 tiles:
+ * q [R][2I] E4M3, qs [R][2I/128] FP32. g, u, dh [R][I] FP32 (G and U are the
+ * forward's pre-activations, recomputed). dgu [R][2I] FP32: the unquantised
+ * [dG | dU] (NULL: not written). I a multiple of 128.
+ */
+MOE_API int moe_swiglu_backward_quant(const float* g, const float* u, const float* dh,
+                              int R, int I, float* dgu, uint8_t* q, float* qs,
+                              void* stream);
+
+/*
+ * moe_quant_1x128_t / moe_quant_128x128_t: wgrad's operands. The rows of x
+ * (row stride ld elements; columns 0..cols-1 are used) form n_groups groups,
+ * rows src_off[g]..src_off[g+1]; group g is transposed into its own
+ * contiguous matrix q_g [cols][K_g] at q + cols * dst_off[g], with K_g =
+ * dst_off[g+1] - dst_off[g] the group's rows rounded up to 128 (the extra
+ * columns are zeros); Ktot = dst_off[n_groups]. Both offset arrays are int32
+ * on the device.
+ *   moe_quant_1x128_t:   x FP32 (x_is_bf16 = 0) or BF16; one scale per 1x128
+ *                        tile along the tokens: s_g [cols][K_g/128] at
+ *                        s + cols * dst_off[g] / 128
+ *   moe_quant_128x128_t: x E4M3 rows with 1x128 scales xs [rows][ld/128]
+ *                        (the forward's FP8 activations), each value
+ *                        dequantised (rounded once to FP32) and requantised in
+ *                        128x128 blocks: s_g [cols/128][K_g/128] at
+ *                        s + (cols/128) * dst_off[g] / 128
+ * cols and Ktot multiples of 128.
+ */
+MOE_API int moe_quant_1x128_t(const void* x, int x_is_bf16, int ld, int cols,
+                      const int32_t* src_off, const int32_t* dst_off, int n_groups,
+                      int Ktot, uint8_t* q, float* s, void* stream);
+MOE_API int moe_quant_128x128_t(const uint8_t* xq, const float* xs, int ld, int cols,
+                        const int32_t* src_off, const int32_t* dst_off, int n_groups,
+                        int Ktot, uint8_t* q, float* s, void* stream);
+
+/*
+ * moe_transpose: for b < batch, dst[b][j][dst_col + i] = src[b][i][j] with
+ * src [batch][rows][cols] and dst [batch][cols][dst_ld]; elements of
+ * elem_bytes = 1 (E4M3 codes) or 4 (FP32 scales). The weights' codes and
+ * block scales for dgrad: a 128x128 block stays one block when transposed,
+ * so the transposed weight is exact.
+ */
+MOE_API int moe_transpose(const void* src, int elem_bytes, int batch, int rows, int cols,
+                  void* dst, int dst_ld, int dst_col, void* stream);
 
 /*
  * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
