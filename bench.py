@@ -420,6 +420,57 @@ def e2e_run(layer, u, e, b, b0, steps, dev, world, cfg):
             "steps": steps, "mode": mode}
 
 
+def backward_run(layer, u, e, b, b0, cfg, dev, peaks, steps=3):
+    """The expert FFNs' FP8 backward on the same layer after one forward, with
+    a seeded BF16 gradient of the expert outputs: dgrad (G and U recomputed,
+    dH, SwiGLU backward, dX; 4 grouped GEMMs) and wgrad (three weight
+    gradients per expert) timed apart with CUDA events, `steps` each."""
+    import torch
+
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    from fine_grained_fp8_sigmoid_b200.backward import ExpertFFNBackward
+    b.copy_(b0)
+    layer.forward(u, e, b, update_bias=False)
+    R = cfg.T * cfg.K_r + cfg.T
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg.seed + 1000)
+    dy = torch.randn(R, cfg.d, generator=g, device=dev).to(torch.bfloat16)
+    bw = ExpertFFNBackward(layer)
+    r = bw.backward(dy)                      # warm-up, both halves
+    idx = torch.cat([layer.sorted_token, torch.arange(cfg.T, dtype=torch.int32, device=dev)])
+    xq = torch.empty(R, cfg.d, dtype=torch.uint8, device=dev)
+    xs = torch.empty(R, cfg.d // 128, dtype=torch.float32, device=dev)
+    B.moe_gather_rows(layer.xq, idx, xq)
+    B.moe_gather_rows(layer.xs, idx, xs)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record(stream)
+    for _ in range(steps):
+        r = bw.backward(dy, wgrad=False)
+    e1.record(stream)
+    for _ in range(steps):
+        bw._wgrad(dy, r["dgu"], xq, xs)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    if B.moe_get_error() != 0:
+        raise RuntimeError("device error word set in the backward")
+    dg_ms, wg_ms = e0.elapsed_time(e1) / steps, e1.elapsed_time(e2) / steps
+    pairs = R                                # (token, expert) rows incl. the shared expert's
+    fl_dg = 2.0 * pairs * cfg.d * cfg.I * 5  # G, U recomputed, dH, and dX (K = 2I: twice)
+    fl_wg = 2.0 * pairs * cfg.d * cfg.I * 3
+    fp8 = 2.0 * peaks["bf16"]
+    del bw, r, dy, xq, xs
+    torch.cuda.empty_cache()
+    return {"what": "expert FFN FP8 backward after one forward, BF16 dY of all routed and shared rows",
+            "steps": steps,
+            "dgrad": {"ms": dg_ms, "tflops": fl_dg / (dg_ms / 1e3) / 1e12,
+                      "frac_of_fp8_burst": fl_dg / (dg_ms / 1e3) / 1e12 / fp8, "gemms": 4},
+            "wgrad": {"ms": wg_ms, "tflops": fl_wg / (wg_ms / 1e3) / 1e12,
+                      "frac_of_fp8_burst": fl_wg / (wg_ms / 1e3) / 1e12 / fp8,
+                      "gemms": 3 * (cfg.N_r + 1), "note": "one GEMM launch per expert and weight"}}
+
+
 def sub_workload(name, args, dev, world, local_rank, peaks):
     """One more workload of the same layer shape, measured in the same run:
     decode (the HBM-bound weight stream) or skew (with its balancing run)."""
@@ -487,6 +538,9 @@ def run_ours(args, rank, world, local_rank):
     layer_tf = layer_flops(cfg) / (ms_step / 1e3) / 1e12
     balance = balance_run(layer, u, e, b, b0) if cfg.name == "skew" else None
     e2e = e2e_run(layer, u, e, b, b0, max(3, K // 2), dev, world, cfg)
+    backward = None
+    if cfg == workloads.CONFIGS[CONFIG_NAME] and not args.no_sub_workloads:
+        backward = backward_run(layer, u, e, b, b0, cfg, dev, peaks)
     del layer, u, e, b, b0
     torch.cuda.empty_cache()
 
@@ -534,6 +588,8 @@ def run_ours(args, rank, world, local_rank):
             "balance": balance,
             "clocks": clocks,
         }
+        if backward is not None:
+            result["backward"] = backward
         result.update(extra)
     return result
 

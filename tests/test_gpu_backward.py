@@ -14,7 +14,6 @@ dX and every expert's weight gradients, <= 2e-3 over all of them (FP32
 rounding alone stays below 1e-5; a wrong scale, operand or transpose gives
 errors of order one).
 """
-import dataclasses
 
 import numpy as np
 import pytest
