@@ -16,13 +16,27 @@
 //
 // Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0     TMA producer: A tile 128 x 128 and B tile 256 x 128 per K block
-//              (128-byte swizzle), 4-stage ring (3 in phase 2).
-//   warp 1     MMA issuer (one thread) and TMEM owner (512 columns = 2 x 256).
-//   warps 2-3  idle (they complete the first warpgroup).
+//              (128-byte swizzle), 4-stage ring (3 in phase 2); with the
+//              gather variant the A rows come straight from the unpermuted
+//              activations by tile::gather4 (four rows per load).
+//   warps 1, 3 MMA issuers (lane 0 of each): warp 1 issues the even K blocks
+//              into TMEM buffer 0, warp 3 the odd ones into buffer 1, so each
+//              waits only on its own buffer's release. Warp 1 owns the TMEM
+//              allocation (512 columns = 2 x 256).
+//   warp 2     idle (it completes the first warpgroup).
 //   warps 4-11 epilogue: warp w reads TMEM lanes 32*(w%4).. (rows), and
 //              (w-4)/4 selects the column half. Each thread keeps 128 FP32
 //              accumulators, so the epilogue warpgroups take 224 registers
 //              per thread and the first warpgroup gives its share back (56).
+//              Each partial is read 32 columns at a time with two reads in
+//              flight, and the buffer is released as soon as the last two
+//              reads have landed in registers, before their FMAs.
+//
+// What paces the K loop: four MMAs of N = 256 take about 513 cycles, but a
+// buffer goes round MMA completion -> read-back of 128 x 256 FP32 values ->
+// FMAs -> release in more than that, and with only two buffers (TMEM holds
+// 512 columns) the round trip is not hidden: a K block takes about 1.2K
+// cycles at d = 7168.
 //
 // Two launches:
 //   phase 1: per tile (group g, 128 rows, 128 intermediate channels n):
