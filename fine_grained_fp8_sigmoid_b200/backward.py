@@ -120,13 +120,17 @@ class ExpertFFNBackward:
         xt, xts = codes(d), torch.empty((d // 128) * (Kt // 128), dtype=f32, device=dev)
         B.moe_quant_128x128_t(xq, xs, src_d, dst_d, xt, xts)
         G = N + 1
-        dw_down = torch.zeros(G, d, I, dtype=f32, device=dev)
-        dw_gate = torch.zeros(G, I, d, dtype=f32, device=dev)
-        dw_up = torch.zeros(G, I, d, dtype=f32, device=dev)
+        # every expert with tokens has its gradients written in full by the
+        # GEMMs; only the others are zero-filled
+        dw_down = torch.empty(G, d, I, dtype=f32, device=dev)
+        dw_gate = torch.empty(G, I, d, dtype=f32, device=dev)
+        dw_up = torch.empty(G, I, d, dtype=f32, device=dev)
         zero = torch.zeros(1, dtype=torch.int32, device=dev)
         for gi in range(G):
             K = int(dst[gi + 1] - dst[gi])
             if K == 0:
+                for w in (dw_down, dw_gate, dw_up):
+                    w[gi].zero_()
                 continue
             o = int(dst[gi])
             act = lambda q, s, rows_: (q[rows_ * o:rows_ * (o + K)].view(rows_, K),

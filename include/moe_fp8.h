@@ -170,7 +170,10 @@ MOE_API int moe_permute(const int32_t* topk_idx, int T, int K_r, int N_r,
  *     rejected with MOE_ERR_UNSUPPORTED (moe_last_error_detail says why).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture. The address is cached per device index for
+ *     the life of the process: after cudaDeviceReset (or any teardown of the
+ *     device's primary context) the cached address is stale, so a process
+ *     that resets a device must not call moe_permute_noalloc on it again.
  *   - All calls share the array: calls that overlap on the GPU (different
  *     streams, or different host threads, on the same device) race and must
  *     be serialised by the caller. Nothing needs clearing between calls.
