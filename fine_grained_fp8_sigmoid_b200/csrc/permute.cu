@@ -109,7 +109,10 @@ __global__ void __launch_bounds__(TOK) scatter_kernel(const int32_t* __restrict_
   const uint32_t lt = (1u << lane_id()) - 1u;
   for (int k = 0; k < K; ++k) {
     const int e = topk[static_cast<size_t>(t) * K + k];
-    if (e < 0 || e >= N_r) continue;
+    if (e < 0 || e >= N_r) {   // the error is recorded by count_kernel
+      inv[static_cast<size_t>(t) * K + k] = -1;
+      continue;
+    }
     int rank = __popc(masks[w * N_r + e] & lt);
     for (int w2 = 0; w2 < w; ++w2) rank += __popc(masks[w2 * N_r + e]);
     const int row = block_base[static_cast<size_t>(blockIdx.x) * N_r + e] + rank;
@@ -120,8 +123,16 @@ __global__ void __launch_bounds__(TOK) scatter_kernel(const int32_t* __restrict_
 
 // One warp per destination row: d bytes of codes as 16-byte vectors, then the
 // d/128 scales.
-__global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__ sorted_token,
-                                                     int P, int T, const uint8_t* __restrict__ xq,
+// Row moves in token order: a warp reads token t's code row (and its
+// scales) once and writes it to the K_r permuted rows inv[t][0..K_r). In
+// permuted order the same token row would be read K_r times, by warps far
+// apart in time, and mostly from DRAM again (L2 does not hold the whole of
+// xq between its uses). The row goes through registers in chunks of up to
+// GV x 16 bytes per lane, all loads of a chunk issued before its stores.
+constexpr int GV = 8;
+
+__global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__ inv, int T, int K,
+                                                     long long P, const uint8_t* __restrict__ xq,
                                                      const float* __restrict__ xs, int d,
                                                      uint8_t* __restrict__ xq_perm,
                                                      float* __restrict__ xs_perm) {
@@ -129,14 +140,33 @@ __global__ void __launch_bounds__(256) gather_kernel(const int32_t* __restrict__
   const int nvec = d / 16;
   const int ns = d / 128;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
-  for (long long p = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); p < P; p += warps) {
-    const int t = sorted_token[p];
-    if (t < 0 || t >= T) continue;  // only after an invalid expert index (error already set)
+  for (long long t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); t < T; t += warps) {
     const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>(t) * d);
-    uint4* dst = reinterpret_cast<uint4*>(xq_perm + static_cast<size_t>(p) * d);
-    for (int i = lane; i < nvec; i += 32) dst[i] = __ldg(src + i);
-    for (int i = lane; i < ns; i += 32)
-      xs_perm[static_cast<size_t>(p) * ns + i] = __ldg(xs + static_cast<size_t>(t) * ns + i);
+    for (int base = 0; base < nvec; base += 32 * GV) {
+      uint4 v[GV];
+#pragma unroll
+      for (int j = 0; j < GV; ++j) {
+        const int i = base + j * 32 + lane;
+        if (i < nvec) v[j] = __ldg(src + i);
+      }
+      for (int k = 0; k < K; ++k) {
+        const long long p = inv[t * K + k];
+        if (p < 0 || p >= P) continue;   // only after an invalid expert index (error already set)
+        uint4* dst = reinterpret_cast<uint4*>(xq_perm + static_cast<size_t>(p) * d);
+#pragma unroll
+        for (int j = 0; j < GV; ++j) {
+          const int i = base + j * 32 + lane;
+          if (i < nvec) dst[i] = v[j];
+        }
+      }
+    }
+    for (int i = lane; i < ns; i += 32) {
+      const float sc = __ldg(xs + static_cast<size_t>(t) * ns + i);
+      for (int k = 0; k < K; ++k) {
+        const long long p = inv[t * K + k];
+        if (p >= 0 && p < P) xs_perm[static_cast<size_t>(p) * ns + i] = sc;
+      }
+    }
   }
 }
 
@@ -183,10 +213,10 @@ extern "C" int moe_permute(const int32_t* topk_idx, int T, int K_r, int N_r, con
   scatter_kernel<<<nb, TOK, sh, s>>>(topk_idx, T, K_r, N_r, block_base, sorted_token, inv);
   if (move_rows) {
     const long long P = static_cast<long long>(T) * K_r;
-    long long blocks = (P + 7) / 8;
-    const long long cap = static_cast<long long>(di.sm_count) * 16;
+    long long blocks = (static_cast<long long>(T) + 7) / 8;       // a warp per token
+    const long long cap = static_cast<long long>(di.sm_count) * 8;  // one resident wave
     if (blocks > cap) blocks = cap;
-    gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(sorted_token, static_cast<int>(P), T, xq, xs, d, xq_perm, xs_perm);
+    gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(inv, T, K_r, P, xq, xs, d, xq_perm, xs_perm);
   }
   return launch_status();
 }

@@ -152,6 +152,9 @@ MOE_API size_t moe_permute_workspace(int T, int N_r);
  *   xq_perm, xs_perm  NULL (when xq is NULL) or [T*K_r][d], [T*K_r][d/128] (out)
  *   workspace    device scratch of moe_permute_workspace(T, N_r) bytes
  * Limits: N_r <= 1024, K_r <= 16, d a multiple of 128.
+ * An expert index outside [0, N_r) records MOE_ERR_INVALID_ARG in the device
+ * error word (moe_get_error); its pair gets inv = -1 and no row, and the rows
+ * that pair would have filled are left unwritten.
  */
 MOE_API int moe_permute(const int32_t* topk_idx, int T, int K_r, int N_r,
                 const uint8_t* xq, const float* xs, int d,
