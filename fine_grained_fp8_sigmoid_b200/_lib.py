@@ -43,6 +43,8 @@ SIGNATURES = {
     "moe_gather_rows": (_i, [_p, _i, _p, _i, _i, _p, _p]),
     "moe_grouped_scaled_gemm_fp8_workspace": (_z, []),
     "moe_grouped_scaled_gemm_fp8": (_i, [_p, _p, _p, _i, _i, _i, _p, _p, _i, _i, _p, _p, _z, _p]),
+    "moe_kgrouped_gemm_fp8_workspace": (_z, []),
+    "moe_kgrouped_gemm_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _z, _p]),
     "moe_swiglu_backward_quant": (_i, [_p, _p, _p, _i, _i, _p, _p, _p, _p]),
     "moe_quant_1x128_t": (_i, [_p, _i, _i, _i, _p, _p, _i, _i, _p, _p, _p]),
     "moe_quant_128x128_t": (_i, [_p, _p, _i, _i, _p, _p, _i, _i, _p, _p, _p]),

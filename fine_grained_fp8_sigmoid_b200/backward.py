@@ -15,7 +15,8 @@ permuted order, then the shared expert's T rows), one call computes
   wgrad  per expert, over its tokens padded to a multiple of 128:
          dW_down = dY^T H,  dW_gate = dG^T X,  dW_up = dU^T X
          (the gradient in 1x128 tiles along the tokens, the forward's X and H
-         requantised in 128x128 blocks)
+         requantised in 128x128 blocks); one K-grouped GEMM launch per weight
+         covers every expert
 
 It reads the forward's state from the MoELayerFP8 (xq, xs, the permutation,
 the intermediate H in the GEMM workspace), so it runs after that forward and
@@ -42,6 +43,7 @@ class ExpertFFNBackward:
         self.wd_t = torch.empty(G, I, d, dtype=torch.uint8, **dev)
         self.sd_t = torch.empty(G, I // 128, d // 128, dtype=torch.float32, **dev)
         self.ws = torch.empty(B.moe_grouped_scaled_gemm_fp8_workspace(), dtype=torch.uint8, **dev)
+        self.kws = torch.empty(B.moe_kgrouped_gemm_fp8_workspace(), dtype=torch.uint8, **dev)
         self.refresh_weights()
 
     def refresh_weights(self):
@@ -97,16 +99,22 @@ class ExpertFFNBackward:
     def _wgrad(self, dy, dgu, xq, xs):
         L = self.layer
         T, d, I, N = L.T, L.d, L.I, L.N_r
-        P, R = T * L.K_r, T * L.K_r + T
+        R = T * L.K_r + T
         dev = L.device
         f32, u8 = torch.float32, torch.uint8
-        # groups: the routed experts, then the shared one; tokens padded to 128
+        # groups: the routed experts, then the shared one; each group's tokens
+        # padded to 128 and laid side by side along K (the transposes are
+        # [cols][Kt], group g in columns dst[g]..dst[g+1])
         src = np.concatenate([L.offsets.cpu().numpy().astype(np.int64), [R]])
         rows = np.diff(src)
         dst = np.concatenate([[0], np.cumsum((rows + 127) // 128 * 128)])
         Kt = int(dst[-1])
         src_d = torch.from_numpy(src.astype(np.int32)).to(dev)
         dst_d = torch.from_numpy(dst.astype(np.int32)).to(dev)
+        G = N + 1
+        dw_down = torch.empty(G, d, I, dtype=f32, device=dev)
+        dw_gate = torch.empty(G, I, d, dtype=f32, device=dev)
+        dw_up = torch.empty(G, I, d, dtype=f32, device=dev)
         codes = lambda cols: torch.empty(cols * Kt, dtype=u8, device=dev)
         dyt, dyts = codes(d), torch.empty(d * Kt // 128, dtype=f32, device=dev)
         B.moe_quant_1x128_t(dy, src_d, dst_d, dyt, dyts)
@@ -119,30 +127,10 @@ class ExpertFFNBackward:
         B.moe_quant_1x128_t(dgu[:, I:], src_d, dst_d, dut, duts)
         xt, xts = codes(d), torch.empty((d // 128) * (Kt // 128), dtype=f32, device=dev)
         B.moe_quant_128x128_t(xq, xs, src_d, dst_d, xt, xts)
-        G = N + 1
-        # every expert with tokens has its gradients written in full by the
-        # GEMMs; only the others are zero-filled
-        dw_down = torch.empty(G, d, I, dtype=f32, device=dev)
-        dw_gate = torch.empty(G, I, d, dtype=f32, device=dev)
-        dw_up = torch.empty(G, I, d, dtype=f32, device=dev)
-        zero = torch.zeros(1, dtype=torch.int32, device=dev)
-        for gi in range(G):
-            K = int(dst[gi + 1] - dst[gi])
-            if K == 0:
-                for w in (dw_down, dw_gate, dw_up):
-                    w[gi].zero_()
-                continue
-            o = int(dst[gi])
-            act = lambda q, s, rows_: (q[rows_ * o:rows_ * (o + K)].view(rows_, K),
-                                       s[rows_ * o // 128:rows_ * (o + K) // 128].view(rows_, K // 128))
-            blk = lambda q, s, rows_: (q[rows_ * o:rows_ * (o + K)].view(1, rows_, K),
-                                       s[(rows_ // 128) * o // 128:(rows_ // 128) * (o + K) // 128].view(1, rows_ // 128, K // 128))
-            a, a_s = act(dyt, dyts, d)
-            b, b_s = blk(ht, hts, I)
-            B.moe_grouped_scaled_gemm_fp8(a, a_s, zero, 0, b, b_s, dw_down[gi], self.ws)
-            b, b_s = blk(xt, xts, d)
-            a, a_s = act(dgt, dgts, I)
-            B.moe_grouped_scaled_gemm_fp8(a, a_s, zero, 0, b, b_s, dw_gate[gi], self.ws)
-            a, a_s = act(dut, duts, I)
-            B.moe_grouped_scaled_gemm_fp8(a, a_s, zero, 0, b, b_s, dw_up[gi], self.ws)
+        act = lambda q, s_, cols: (q.view(cols, Kt), s_.view(cols, Kt // 128))
+        blk = lambda q, s_, cols: (q.view(cols, Kt), s_.view(cols // 128, Kt // 128))
+        # one launch per weight: every expert over its own token range
+        B.moe_kgrouped_gemm_fp8(*act(dyt, dyts, d), *blk(ht, hts, I), dst_d, dw_down, self.kws)
+        B.moe_kgrouped_gemm_fp8(*act(dgt, dgts, I), *blk(xt, xts, d), dst_d, dw_gate, self.kws)
+        B.moe_kgrouped_gemm_fp8(*act(dut, duts, I), *blk(xt, xts, d), dst_d, dw_up, self.kws)
         return dict(dw_gate=dw_gate, dw_up=dw_up, dw_down=dw_down)

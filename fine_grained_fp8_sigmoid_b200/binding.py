@@ -270,6 +270,28 @@ def moe_grouped_scaled_gemm_fp8(a, a_s, offsets, P, b, b_s, c, workspace, stream
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def moe_kgrouped_gemm_fp8_workspace():
+    return int(_lib.load().moe_kgrouped_gemm_fp8_workspace())
+
+
+def moe_kgrouped_gemm_fp8(a, a_s, b, b_s, kofs, c, workspace, stream=None):
+    """c[g] = a[:, K_g] b[:, K_g]^T for K_g = kofs[g]..kofs[g+1]: a [M][K]
+    E4M3 (1x128 scales a_s [M][K/128]), b [N][K] E4M3 (128x128 scales b_s
+    [N/128][K/128]), kofs [G+1] int32, c [G][M][N] FP32."""
+    M, K = a.shape
+    N = b.shape[0]
+    G = kofs.shape[0] - 1
+    _want(a, torch.uint8, (M, K), "a")
+    _want(a_s, torch.float32, (M, K // 128), "a_s")
+    _want(b, torch.uint8, (N, K), "b")
+    _want(b_s, torch.float32, (N // 128, K // 128), "b_s")
+    _want(kofs, torch.int32, (G + 1,), "kofs")
+    _want(c, torch.float32, (G, M, N), "c")
+    check("moe_kgrouped_gemm_fp8", _lib.load().moe_kgrouped_gemm_fp8(
+        _ptr(a), _ptr(a_s), _ptr(b), _ptr(b_s), _ptr(kofs), G, M, N, K, _ptr(c),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
 def moe_swiglu_backward_quant(g, u, dh, dgu, q, qs, stream=None):
     R, I = g.shape
     for t, n in ((g, "g"), (u, "u"), (dh, "dh")):
@@ -289,8 +311,9 @@ def _ld(x):
 
 def moe_quant_1x128_t(x, src_off, dst_off, q, s, stream=None):
     """x [rows][cols] FP32 or BF16 (a column slice of a wider row-major tensor
-    is allowed) -> per group g a [cols][K_g] block of q (flat, cols * Ktot
-    bytes) and a [cols][K_g/128] block of s (flat)."""
+    is allowed) -> its per-group transpose q [cols][Ktot] (flat, cols * Ktot
+    bytes; group g in columns dst_off[g]..dst_off[g+1]) and s [cols][Ktot/128]
+    (flat)."""
     if x.dtype not in (torch.float32, torch.bfloat16):
         raise ValueError("x must be FP32 or BF16")
     cols = x.shape[1]
@@ -306,8 +329,9 @@ def moe_quant_1x128_t(x, src_off, dst_off, q, s, stream=None):
 
 
 def moe_quant_128x128_t(xq, xs, src_off, dst_off, q, s, stream=None):
-    """xq [rows][cols] E4M3 with 1x128 scales xs -> per group g a [cols][K_g]
-    block of q (flat) in 128x128 blocks, scales [cols/128][K_g/128] (flat)."""
+    """xq [rows][cols] E4M3 with 1x128 scales xs -> its per-group transpose
+    q [cols][Ktot] (flat) in 128x128 blocks, scales [cols/128][Ktot/128]
+    (flat)."""
     rows, cols = xq.shape
     Ktot = q.numel() // cols
     n = src_off.shape[0] - 1

@@ -93,64 +93,128 @@ __device__ __forceinline__ int block_group(const int32_t* dst_off, int n_groups,
   return lo;
 }
 
-// One block of 128 threads per (128 tokens, 128 columns): the tile is staged
-// in shared memory as [token][column]; thread c then owns column c: its 128
-// token values form one 1x128 tile of the transposed tensor (KIND 0: FP32
-// input, KIND 1: BF16 input; a scale per column and token block) or belong to
-// one 128x128 block (KIND 2: FP8 input with 1x128 scales; one scale for the
-// whole tile).
+// One block of 256 threads per (128 tokens, 128 columns). The tile is read
+// with 16-byte loads (thread t: token t/2, half t%2 of the columns) and
+// staged in shared memory as [token][column] in the input's own type (so
+// that several blocks fit an SM); thread t then owns column t%128 over tokens
+// (t/128)*64..+64: those values belong to one 1x128 tile of the transposed
+// tensor (KIND 0: FP32 input, KIND 1: BF16 input; a scale per column and
+// token block, the two halves' max-abs combined) or to one 128x128 block
+// (KIND 2: FP8 input with 1x128 scales, each value dequantised and rounded
+// once to FP32; one scale for the whole tile). The codes are staged again as
+// [column][token] rows and leave as 128-byte row segments.
+template <int KIND> struct QtStage;
+template <> struct QtStage<0> { using E = float;    static constexpr int LD = 132; };  // elements per row
+template <> struct QtStage<1> { using E = uint16_t; static constexpr int LD = 136; };
+template <> struct QtStage<2> { using E = uint8_t;  static constexpr int LD = 144; };
+constexpr int QT_OUT_LD = 144;    // bytes per staged output row (16-byte aligned, spreads the banks)
+
 template <int KIND>
-__global__ void __launch_bounds__(128) quant_t_kernel(const void* __restrict__ x, const float* __restrict__ xs,
+constexpr size_t qt_smem_bytes() {
+  return 128 * QtStage<KIND>::LD * sizeof(typename QtStage<KIND>::E) + 128 * QT_OUT_LD;
+}
+
+template <int KIND>
+__device__ __forceinline__ float qt_value(const typename QtStage<KIND>::E v, float sx) {
+  if (KIND == 0) return v;
+  if (KIND == 1) return bf16_bits_to_float(v);
+  __half_raw hr = __nv_cvt_fp8_to_halfraw(v, __NV_E4M3);
+  return __half2float(__half(hr)) * sx;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(256) quant_t_kernel(const void* __restrict__ x, const float* __restrict__ xs,
                                                       int ld, int cols, const int32_t* __restrict__ src_off,
                                                       const int32_t* __restrict__ dst_off, int n_groups, int Ktot,
                                                       uint8_t* __restrict__ q, float* __restrict__ s) {
-  extern __shared__ float tile[];                    // [128][129]
-  __shared__ float red[4];
-  const int p = blockIdx.x;                          // token block of the output's K
-  const int cb = blockIdx.y;                         // column block
+  using E = typename QtStage<KIND>::E;
+  constexpr int LD = QtStage<KIND>::LD;
+  constexpr int VEC = 16 / sizeof(E);                 // elements per 16-byte load
+  extern __shared__ __align__(16) uint8_t qt_raw[];
+  E* tile = reinterpret_cast<E*>(qt_raw);             // [128][LD]
+  uint8_t* out = qt_raw + 128 * LD * sizeof(E);       // [128][QT_OUT_LD]
+  __shared__ float red[2][128];
+  __shared__ float bred[8];
+  __shared__ float rsx[128];                          // KIND 2: each token row's 1x128 scale
+  const int p = blockIdx.x;                           // token block of the output's K
+  const int cb = blockIdx.y;                          // column block
   const int g = block_group(dst_off, n_groups, p * 128);
-  const int d0 = __ldg(dst_off + g), Kg = __ldg(dst_off + g + 1) - d0;   // the group's padded token count
+  const int d0 = __ldg(dst_off + g);
   const int first = __ldg(src_off + g) + (p * 128 - d0);
   const int live = max(0, min(128, __ldg(src_off + g + 1) - first));
-  const int c = threadIdx.x;
-  for (int t = 0; t < 128; ++t) {
-    float v = 0.0f;
-    if (t < live) {
-      const size_t at = static_cast<size_t>(first + t) * ld + cb * 128 + c;
-      if (KIND == 0) {
-        v = __ldg(static_cast<const float*>(x) + at);
-      } else if (KIND == 1) {
-        v = bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(x) + at));
-      } else {   // FP8 row with 1x128 scales: the forward's value, rounded once to FP32
-        const uint8_t code = static_cast<const uint8_t*>(x)[at];
-        __half_raw hr = __nv_cvt_fp8_to_halfraw(code, __NV_E4M3);
-        v = __half2float(__half(hr)) * __ldg(xs + static_cast<size_t>(first + t) * (ld / 128) + cb);
-      }
+  const int tid = threadIdx.x;
+  {
+    const int r = tid >> 1, h = tid & 1;
+    uint4* trow = reinterpret_cast<uint4*>(tile + r * LD + h * 64);
+    constexpr int NV = 64 / VEC;
+    if (r < live) {
+      const size_t at = static_cast<size_t>(first + r) * ld + cb * 128 + h * 64;
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const E*>(x) + at);
+      uint4 v[NV];
+#pragma unroll
+      for (int i = 0; i < NV; ++i) v[i] = __ldg(src + i);
+#pragma unroll
+      for (int i = 0; i < NV; ++i) trow[i] = v[i];
+      if (KIND == 2 && h == 0) rsx[r] = __ldg(xs + static_cast<size_t>(first + r) * (ld / 128) + cb);
+    } else {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) trow[i] = make_uint4(0, 0, 0, 0);
+      if (KIND == 2 && h == 0) rsx[r] = 0.0f;
     }
-    tile[t * 129 + c] = v;
   }
   __syncthreads();
+  const int c = tid & 127, th = tid >> 7;
+  const E* tcol = tile + th * 64 * LD + c;
+  const float* sxc = rsx + th * 64;
   float amax = 0.0f;
-  for (int t = 0; t < 128; ++t) amax = fmaxf(amax, fabsf(tile[t * 129 + c]));
-  if (KIND == 2) {
+#pragma unroll 8
+  for (int t = 0; t < 64; ++t) amax = fmaxf(amax, fabsf(qt_value<KIND>(tcol[t * LD], KIND == 2 ? sxc[t] : 0.0f)));
+  if (KIND != 2) {
+    red[th][c] = amax;
+    __syncthreads();
+    amax = fmaxf(red[0][c], red[1][c]);
+  } else {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane_id() == 0) red[c >> 5] = amax;
+    if (lane_id() == 0) bred[tid >> 5] = amax;
     __syncthreads();
-    amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    amax = bred[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) amax = fmaxf(amax, bred[i]);
   }
   const float sc = tile_scale(amax);
-  // group-major output: group g is the contiguous matrix [cols][Kg] at
-  // cols * d0, so that one GEMM reads it with its own row stride
-  uint8_t* qrow = q + static_cast<size_t>(cols) * d0 + static_cast<size_t>(cb * 128 + c) * Kg + (p * 128 - d0);
-  for (int t = 0; t < 128; t += 4) {
-    const uint32_t w = e4m3x2(__fdiv_rn(tile[t * 129 + c], sc), __fdiv_rn(tile[(t + 1) * 129 + c], sc)) |
-                       (e4m3x2(__fdiv_rn(tile[(t + 2) * 129 + c], sc), __fdiv_rn(tile[(t + 3) * 129 + c], sc)) << 16);
-    *reinterpret_cast<uint32_t*>(qrow + t) = w;
+  uint8_t* orow = out + c * QT_OUT_LD + th * 64;
+#pragma unroll
+  for (int t = 0; t < 64; t += 16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tt = t + 4 * k + e;
+        v[e] = __fdiv_rn(qt_value<KIND>(tcol[tt * LD], KIND == 2 ? sxc[tt] : 0.0f), sc);
+      }
+      w[k] = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
+    }
+    *reinterpret_cast<uint4*>(orow + t) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  const int pg = p - d0 / 128;              // token block within the group
-  if (KIND != 2) s[static_cast<size_t>(cols) * (d0 / 128) + static_cast<size_t>(cb * 128 + c) * (Kg / 128) + pg] = sc;
-  else if (c == 0) s[static_cast<size_t>(cols / 128) * (d0 / 128) + static_cast<size_t>(cb) * (Kg / 128) + pg] = sc;
+  if (KIND != 2) {
+    if (th == 0) s[static_cast<size_t>(cb * 128 + c) * (Ktot / 128) + p] = sc;
+  } else if (tid == 0) {
+    s[static_cast<size_t>(cb) * (Ktot / 128) + p] = sc;
+  }
+  __syncthreads();
+  // output [cols][Ktot]: group g holds columns d0 .. d0 + K_g of every row,
+  // so one K-grouped GEMM reads all groups through one tensor map; eight
+  // threads write one row's 128 bytes of this token block
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int row = pass * 32 + (tid >> 3), chunk = tid & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(out + row * QT_OUT_LD + chunk * 16);
+    *reinterpret_cast<uint4*>(q + static_cast<size_t>(cb * 128 + row) * Ktot + static_cast<size_t>(p) * 128 +
+                              chunk * 16) = v;
+  }
 }
 
 // dst[b][j][dst_col + i] = src[b][i][j], 32 x 32 tiles through shared memory.
@@ -208,19 +272,21 @@ static int quant_t(int kind, const void* x, const float* xs, int ld, int cols, c
   MOE_CHECK_ARG(x && src_off && dst_off && q && s && (kind != 2 || xs));
   DeviceInfo di;
   if (int st = device_info(&di)) return st;
-  const size_t sh = 128 * 129 * sizeof(float);
+  const size_t esz = kind == 0 ? 4 : kind == 1 ? 2 : 1;
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(x) % 16 == 0 && (static_cast<size_t>(ld) * esz) % 16 == 0 &&
+                reinterpret_cast<uintptr_t>(q) % 16 == 0);
   dim3 grid(Ktot / 128, cols / 128);
   cudaStream_t st = as_stream(stream);
-  auto launch = [&](auto kern) -> int {
+  auto launch = [&](auto kern, size_t sh) -> int {
     if (int e = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sh)),
                             "quant_t smem attribute"))
       return e;
-    kern<<<grid, 128, sh, st>>>(x, xs, ld, cols, src_off, dst_off, n_groups, Ktot, q, s);
+    kern<<<grid, 256, sh, st>>>(x, xs, ld, cols, src_off, dst_off, n_groups, Ktot, q, s);
     return launch_status("transposed quantisation");
   };
-  if (kind == 0) return launch(bwd::quant_t_kernel<0>);
-  if (kind == 1) return launch(bwd::quant_t_kernel<1>);
-  return launch(bwd::quant_t_kernel<2>);
+  if (kind == 0) return launch(bwd::quant_t_kernel<0>, bwd::qt_smem_bytes<0>());
+  if (kind == 1) return launch(bwd::quant_t_kernel<1>, bwd::qt_smem_bytes<1>());
+  return launch(bwd::quant_t_kernel<2>, bwd::qt_smem_bytes<2>());
 }
 
 extern "C" int moe_quant_1x128_t(const void* x, int x_is_bf16, int ld, int cols, const int32_t* src_off,

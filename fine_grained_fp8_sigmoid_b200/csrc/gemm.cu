@@ -125,6 +125,10 @@ struct Args {
   float* y_shared;
   int* tile_counter;         // zeroed before the launch; tiles past the first wave are claimed from it
   const int32_t* sorted_token;  // non-null: routed rows are read from xq/xs at these tokens (no xq_perm)
+  // K-grouped (phase 2 only): N_r + 1 groups share A's T rows and B's rows;
+  // group g contracts over K elements offsets[g]..offsets[g+1] (multiples of
+  // 128; I = the total K) and writes output rows g*T..g*T+T
+  int kgrouped;
 };
 
 template <int STAGES, int TAB_KB>
@@ -177,6 +181,8 @@ __device__ __forceinline__ int find_group(const int* start, int G, int t) {
 
 struct Tile {
   int g, m, n, rows, row0;  // rows of the group; row0 = first row of the group in its A tensor
+  int orow0;                // first output row of the group (row0 unless K-grouped)
+  int k0, kb;               // the tile's K blocks: k0 .. k0 + kb
   int mrows;                // narrow tile: its rows (1..narrow_max, the whole group)
   bool shared, narrow;
 };
@@ -189,6 +195,25 @@ __device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, i
   const int local = t - sm.tile_start[tl.g];
   tl.m = local / n_tiles;
   tl.n = local - tl.m * n_tiles;
+  tl.k0 = 0;
+  tl.kb = (PHASE == 1 ? a.d : a.I) / BK;
+  if (PHASE == 2 && a.kgrouped) {
+    tl.shared = false;
+    tl.rows = a.T;
+    tl.row0 = 0;
+    tl.orow0 = tl.g * a.T;
+    const int lo = sm.off[tl.g], hi = sm.off[tl.g + 1];
+    if (lo < 0 || hi < lo || hi > a.I || lo % BK != 0 || hi % BK != 0) {
+      set_device_error(MOE_ERR_INVALID_ARG);   // every role decodes the same: no K blocks
+      tl.kb = 0;
+    } else {
+      tl.k0 = lo / BK;
+      tl.kb = (hi - lo) / BK;
+    }
+    tl.mrows = 0;
+    tl.narrow = false;
+    return tl;
+  }
   tl.shared = tl.g == a.N_r;
   if (tl.shared) {
     tl.rows = a.T;
@@ -197,6 +222,7 @@ __device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, i
     tl.row0 = sm.off[tl.g];
     tl.rows = sm.off[tl.g + 1] - tl.row0;
   }
+  tl.orow0 = tl.row0;
   tl.mrows = narrow_part(tl.rows, a.narrow_max);  // a narrow group has one row tile
   tl.narrow = tl.mrows > 0;
   return tl;
@@ -457,10 +483,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i <= a.N_r; i += THREADS) sm.off[i] = a.offsets[i];
+  const bool kg = PHASE == 2 && a.kgrouped;
+  for (int i = threadIdx.x; i <= (kg ? G : a.N_r); i += THREADS) sm.off[i] = a.offsets[i];
   __syncthreads();
   for (int g = threadIdx.x; g < G; g += THREADS) {
-    const int rows = g == a.N_r ? a.T : sm.off[g + 1] - sm.off[g];
+    const int rows = (kg || g == a.N_r) ? a.T : sm.off[g + 1] - sm.off[g];
     sm.tile_start[g] = ((rows + BM - 1) / BM) * n_tiles;
   }
   __syncthreads();
@@ -545,21 +572,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int i = 0; i < 4; ++i) tok[i] = __ldg(a.sorted_token + min(arow + 4 * lane + i, last));
         }
         const uint32_t stage_bytes = gather ? STAGE_BYTES - A_BYTES + n_g4 * 4 * BK : STAGE_BYTES;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < tl.kb; ++kb) {
+          const int kx = (tl.k0 + kb) * BK;
           int okw = 1;
           uint8_t* dst = tiles + stage * STAGE_BYTES;
           if (lane == 0) {
             okw = mbar_wait(&sm.empty[stage], phase ^ 1, abort) ? 1 : 0;
             if (okw) {
               mbar_arrive_expect_tx(&sm.full[stage], stage_bytes);
-              if (!gather) tma_load_2d(dst, am, &sm.full[stage], kb * BK, arow);
+              if (!gather) tma_load_2d(dst, am, &sm.full[stage], kx, arow);
               if (PHASE == 1) {
                 const int wrow = tl.g * a.I + tl.n * 128;
-                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
-                tma_load_2d_hint(dst + A_BYTES + B_BYTES / 2, &tm_b1, &sm.full[stage], kb * BK, wrow, pol_w);
+                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kx, wrow, pol_w);
+                tma_load_2d_hint(dst + A_BYTES + B_BYTES / 2, &tm_b1, &sm.full[stage], kx, wrow, pol_w);
               } else {
-                const int wrow = tl.g * a.d + tl.n * BN;
-                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kb * BK, wrow, pol_w);
+                const int wrow = (kg ? 0 : tl.g * a.d) + tl.n * BN;
+                tma_load_2d_hint(dst + A_BYTES, &tm_b0, &sm.full[stage], kx, wrow, pol_w);
               }
               armed[stage] = phase;
             }
@@ -567,7 +595,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           okw = __shfl_sync(0xffffffffu, okw, 0);   // also orders the copies after the expected bytes
           if (!okw) break;
           if (gather && lane < n_g4)
-            tma_gather4(dst + lane * 4 * BK, &tm_xg, &sm.full[stage], kb * BK, tok[0], tok[1], tok[2], tok[3]);
+            tma_gather4(dst + lane * 4 * BK, &tm_xg, &sm.full[stage], kx, tok[0], tok[1], tok[2], tok[3]);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -615,7 +643,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // 128 of the buffer), the tile's first N = rows rounded up to 16 token
         // rows of the A stage are N
         const uint32_t idesc_n = make_idesc(0, 0, 128, (tl.mrows + 15) & ~15);
-        for (int kb = 0; kb < KB; ++kb, kpar ^= 1) {
+        for (int kb = 0; kb < tl.kb; ++kb, kpar ^= 1) {
           if (kpar != static_cast<uint32_t>(j)) continue;
           // the operands usually land well before the partial buffer is free:
           // check them first, so that only the buffer's wait sits between the
@@ -706,26 +734,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           sa_ptr = a.xs + static_cast<size_t>(valid ? __ldg(a.sorted_token + grow) : 0) * KBd;
         sb0 = a.s_gate + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
         sb1 = a.s_up + static_cast<size_t>(tl.g * KBi + tl.n) * KBd;
-      } else {
-        sa_ptr = a.Hs + static_cast<size_t>(grow) * KBi;
-        sb0 = a.s_down + static_cast<size_t>(tl.g * KBd + tl.n * 2 + half) * KBi;
+      } else {   // K-grouped: one B for all groups, the tile's K range from k0
+        sa_ptr = a.Hs + static_cast<size_t>(grow) * KBi + tl.k0;
+        sb0 = a.s_down + static_cast<size_t>((kg ? 0 : tl.g * KBd) + tl.n * 2 + half) * KBi + tl.k0;
         sb1 = sb0;
       }
+      const int KBt = tl.kb;
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
       // The row's activation scale (a different cache line for every
       // thread) is loaded two K blocks ahead, the weight block's scales (one
       // line for the whole CTA) one block ahead.
-      float sa_n = valid ? __ldg(sa_ptr) : 0.0f;
-      float sa_n2 = (valid && KB > 1) ? __ldg(sa_ptr + 1) : 0.0f;
-      float s0_n = __ldg(sb0), s1_n = __ldg(sb1);
+      float sa_n = (valid && KBt > 0) ? __ldg(sa_ptr) : 0.0f;
+      float sa_n2 = (valid && KBt > 1) ? __ldg(sa_ptr + 1) : 0.0f;
+      float s0_n = KBt > 0 ? __ldg(sb0) : 0.0f, s1_n = KBt > 0 ? __ldg(sb1) : 0.0f;
       bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < KBt; ++kb) {
         const float sa = sa_n, s0 = s0_n, s1 = s1_n;
         sa_n = sa_n2;
-        if (kb + 2 < KB) sa_n2 = valid ? __ldg(sa_ptr + kb + 2) : 0.0f;
-        if (kb + 1 < KB) {
+        if (kb + 2 < KBt) sa_n2 = valid ? __ldg(sa_ptr + kb + 2) : 0.0f;
+        if (kb + 1 < KBt) {
           s0_n = __ldg(sb0 + kb + 1);
           s1_n = __ldg(sb1 + kb + 1);
         }
@@ -817,7 +846,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int col0 = tl.n * BN + half * 128;
         if (nvalid == Y_BOX) {
           const CUtensorMap* ym = tl.shared ? &tm_ys : &tm_y;
-          const int ytop = tl.shared ? row_first : tl.row0 + row_first;
+          const int ytop = tl.shared ? row_first : tl.orow0 + row_first;
           uint8_t* wstage = staging + ew * 2 * Y_BOX_BYTES;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -838,7 +867,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else if (valid) {
           float* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
-                                  : a.y_perm + static_cast<size_t>(tl.row0 + rr) * a.d;
+                                  : a.y_perm + static_cast<size_t>(tl.orow0 + rr) * a.d;
           float4* dst = reinterpret_cast<float4*>(yrow + col0);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -957,7 +986,7 @@ static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int3
   // schedule at T = 8192 with 39 groups of <= 64 rows: +4.2 GB of DRAM reads).
   const bool narrow = narrow_enabled(d, I) && P <= static_cast<long long>(NMAX) * N_r;
 
-  Args args;
+  Args args{};
   args.offsets = offsets;
   args.N_r = N_r;
   args.T = T;
@@ -1095,4 +1124,60 @@ extern "C" int moe_grouped_scaled_gemm_fp8(const uint8_t* a, const float* a_s, c
     return st;
   k2<<<grid, THREADS, sm2, s>>>(tmA, tmA, tmB, tmB, tmC, tmCs, tmA, args);
   return launch_status("scaled GEMM launch");
+}
+
+// K-grouped scaled GEMM on the same kernel: per group g,
+// C_g = A[:, K_g] B[:, K_g]^T over the group's own K range K_g =
+// kofs[g]..kofs[g+1]. The backward's weight gradients have this form: an
+// expert's gradient contracts over that expert's tokens.
+extern "C" size_t moe_kgrouped_gemm_fp8_workspace(void) { return 256; }
+
+extern "C" int moe_kgrouped_gemm_fp8(const uint8_t* a, const float* a_s, const uint8_t* b, const float* b_s,
+                                     const int32_t* kofs, int G, int M, int N, int K_total, float* c,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  using namespace moe;
+  using namespace moe::gg;
+  MOE_CHECK_ARG(G >= 1 && M >= 0 && N >= 0 && K_total >= 0);
+  MOE_CHECK_SUPPORTED(G <= MAX_GROUPS - 1 && M % BM == 0 && N % BN == 0 && K_total % BK == 0);
+  MOE_CHECK_SUPPORTED(static_cast<long long>(G) * M < (1LL << 31) && K_total < (1 << 30));
+  if (M == 0 || N == 0) return MOE_OK;
+  MOE_CHECK_ARG(c && workspace && ws_bytes >= moe_kgrouped_gemm_fp8_workspace());
+  MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(workspace) % 16 == 0 && reinterpret_cast<uintptr_t>(c) % 16 == 0);
+  cudaStream_t s = as_stream(stream);
+  if (K_total == 0)   // every group is empty: the products are zero
+    return cuda_status(cudaMemsetAsync(c, 0, static_cast<size_t>(G) * M * N * sizeof(float), s),
+                       "K-grouped GEMM: zero output");
+  MOE_CHECK_ARG(a && a_s && b && b_s && kofs);
+  DeviceInfo di;
+  if (int st = device_info(&di)) return st;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUtensorMap tmA, tmB, tmC;
+  if (int st = make_tmap_2d(&tmA, a, U8, 1, M, K_total, BM, BK)) return st;
+  if (int st = make_tmap_2d(&tmB, b, U8, 1, N, K_total, BN, BK)) return st;
+  if (int st = make_tmap_y(&tmC, c, static_cast<uint64_t>(G) * M, N)) return st;
+  Args args{};
+  args.offsets = kofs;
+  args.N_r = G - 1;
+  args.T = M;
+  args.P = 0;
+  args.d = N;          // the down kernel's output width
+  args.I = K_total;    // its contraction (all groups' K ranges)
+  args.Hs = const_cast<float*>(a_s);
+  args.s_down = b_s;
+  args.y_perm = c;
+  args.y_shared = c;
+  args.narrow_max = 0;
+  args.sorted_token = nullptr;
+  args.kgrouped = 1;
+  args.tile_counter = static_cast<int*>(workspace);
+  if (int st = cuda_status(cudaMemsetAsync(workspace, 0, sizeof(int), s), "K-grouped GEMM: tile counter")) return st;
+  const long long tiles = static_cast<long long>(G) * (M / BM) * (N / BN);
+  const int grid = static_cast<int>(tiles < di.sm_count ? tiles : di.sm_count);
+  auto k2 = grouped_gemm_kernel<2>;
+  constexpr size_t sm2 = smem_bytes<2>();
+  if (int st = cuda_status(cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2)),
+                           "smem attribute (K-grouped GEMM)"))
+    return st;
+  k2<<<grid, THREADS, sm2, s>>>(tmA, tmA, tmB, tmB, tmC, tmC, tmA, args);
+  return launch_status("K-grouped GEMM launch");
 }

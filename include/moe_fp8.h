@@ -340,6 +340,29 @@ MOE_API int moe_grouped_scaled_gemm_fp8(const uint8_t* a, const float* a_s,
                          float* c, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * moe_kgrouped_gemm_fp8: for each group g < G, over its own K range
+ * K_g = kofs[g] .. kofs[g+1] (elements),
+ *   C_g = A[:, K_g] B[:, K_g]^T     (C_g = c + g * M * N, [M][N] FP32)
+ * with FP32 promotion per 128-wide K block, on the grouped GEMM kernel. The
+ * backward's weight gradients have this form (each expert contracts over its
+ * own tokens), and one launch covers every expert.
+ *   a, a_s   [M][K_total] E4M3, [M][K_total/128] FP32 (1x128 tiles along K)
+ *   b, b_s   [N][K_total] E4M3, [N/128][K_total/128] FP32 (128x128 blocks)
+ *   kofs     [G+1] int32 (device): non-decreasing multiples of 128 within
+ *            [0, K_total]; a group with an empty range gets C_g = 0. A range
+ *            that breaks this records MOE_ERR_INVALID_ARG in the device
+ *            error word and its C_g is written as zero.
+ *   workspace  moe_kgrouped_gemm_fp8_workspace() bytes (a tile counter)
+ * Limits: M a multiple of 128, N a multiple of 256, K_total a multiple of
+ * 128, G <= 1024.
+ */
+MOE_API size_t moe_kgrouped_gemm_fp8_workspace(void);
+MOE_API int moe_kgrouped_gemm_fp8(const uint8_t* a, const float* a_s, const uint8_t* b,
+                          const float* b_s, const int32_t* kofs, int G, int M, int N,
+                          int K_total, float* c, void* workspace, size_t ws_bytes,
+                          void* stream);
+
+/*
  * moe_swiglu_backward_quant: for rows r < R and columns i < I,
  *   dG = dH U silu'(G),  dU = dH silu(G),  silu'(x) = s(x)(1 + x(1 - s(x)))
  * with s the sigmoid, then [dG | dU] ([R][2I]) quantised in 1x128 tiles:
@@ -354,20 +377,19 @@ MOE_API int moe_swiglu_backward_quant(const float* g, const float* u, const floa
 /*
  * moe_quant_1x128_t / moe_quant_128x128_t: wgrad's operands. The rows of x
  * (row stride ld elements; columns 0..cols-1 are used) form n_groups groups,
- * rows src_off[g]..src_off[g+1]; group g is transposed into its own
- * contiguous matrix q_g [cols][K_g] at q + cols * dst_off[g], with K_g =
- * dst_off[g+1] - dst_off[g] the group's rows rounded up to 128 (the extra
- * columns are zeros); Ktot = dst_off[n_groups]. Both offset arrays are int32
- * on the device.
+ * rows src_off[g]..src_off[g+1]. The output is the transpose q [cols][Ktot]
+ * E4M3 with Ktot = dst_off[n_groups]: group g fills its columns
+ * dst_off[g] .. dst_off[g+1] of every row, its rows rounded up to a multiple
+ * of 128 (the extra columns are zeros). Both offset arrays are int32 on the
+ * device; dst_off[g] are multiples of 128.
  *   moe_quant_1x128_t:   x FP32 (x_is_bf16 = 0) or BF16; one scale per 1x128
- *                        tile along the tokens: s_g [cols][K_g/128] at
- *                        s + cols * dst_off[g] / 128
+ *                        tile along the tokens: s [cols][Ktot/128]
  *   moe_quant_128x128_t: x E4M3 rows with 1x128 scales xs [rows][ld/128]
  *                        (the forward's FP8 activations), each value
  *                        dequantised (rounded once to FP32) and requantised in
- *                        128x128 blocks: s_g [cols/128][K_g/128] at
- *                        s + (cols/128) * dst_off[g] / 128
- * cols and Ktot multiples of 128.
+ *                        128x128 blocks: s [cols/128][Ktot/128]
+ * cols and Ktot multiples of 128. A 128-wide token block never spans two
+ * groups, so every tile and block holds one expert's tokens.
  */
 MOE_API int moe_quant_1x128_t(const void* x, int x_is_bf16, int ld, int cols,
                       const int32_t* src_off, const int32_t* dst_off, int n_groups,

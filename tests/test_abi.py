@@ -46,6 +46,8 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
+    assert lib.moe_kgrouped_gemm_fp8_workspace() >= 4
+    assert lib.moe_grouped_scaled_gemm_fp8_workspace() >= 4
     assert lib.moe_permute_workspace(8192, 256) == 2 * 32 * 256 * 4
     assert lib.moe_permute_workspace(0, 256) == 0
     rows = 8192 * 8 + 8192
@@ -81,6 +83,11 @@ def test_host_side_argument_checks(lib):
                                     N, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_grouped_gemm_fp8(N, N, N, 8, 2, N, N, 4, N, N, N, N, N, N, 256, 100,
                                     N, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
+    # K-grouped GEMM: M not a multiple of 128, N not a multiple of 256, G = 0
+    assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 4, 100, 256, 128, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 4, 128, 384, 128, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
+    assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 0, 128, 256, 128, N, N, 0, s) == _lib.MOE_ERR_INVALID_ARG
+    assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 4, 128, 256, 128, N, N, 0, s) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_combine(N, N, N, N, N, 4, 2, 12, N, s) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_bias_update(N, N, 8, 4, 2, ctypes.c_float(0.001), N, s) == _lib.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_wait_timeout(0, s) == _lib.MOE_ERR_INVALID_ARG

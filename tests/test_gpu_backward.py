@@ -75,7 +75,9 @@ def test_transposed_quantisation_bit_exact(lib, rows, cols):
     sb = torch.empty((cols // 128) * (Kt // 128), device="cuda")
     B.moe_quant_128x128_t(torch.from_numpy(xq).cuda(), torch.from_numpy(xs).float().cuda(), sd, dd, qb, sb)
     torch.cuda.synchronize()
-    q, s, qb, sb = q.cpu().numpy(), s.cpu().double().numpy(), qb.cpu().numpy(), sb.cpu().double().numpy()
+    # layout [cols][Kt]: group g in columns dst[g]..dst[g+1] of every row
+    q, s = q.cpu().numpy().reshape(cols, Kt), s.cpu().double().numpy().reshape(cols, Kt // 128)
+    qb, sb = qb.cpu().numpy().reshape(cols, Kt), sb.cpu().double().numpy().reshape(cols // 128, Kt // 128)
     for g in range(len(rows)):
         K = int(dst[g + 1] - dst[g])
         if K == 0:
@@ -83,13 +85,12 @@ def test_transposed_quantisation_bit_exact(lib, rows, cols):
         o = int(dst[g])
         xg = _pad(x[src[g]:src[g + 1]], K).T
         rq, rs = O.quant_1x128(xg)
-        assert np.array_equal(q[cols * o:cols * (o + K)].reshape(cols, K), rq), g
-        assert np.array_equal(s[cols * o // 128:cols * (o + K) // 128].reshape(cols, K // 128), rs), g
+        assert np.array_equal(q[:, o:o + K], rq), g
+        assert np.array_equal(s[:, o // 128:(o + K) // 128], rs), g
         hg = _pad(O.dequant_1x128(xq, xs)[src[g]:src[g + 1]], K).T
         bq, bs = O.quant_128x128(round_fp32(hg))
-        assert np.array_equal(qb[cols * o:cols * (o + K)].reshape(cols, K), bq), g
-        nb = (cols // 128) * o // 128
-        assert np.array_equal(sb[nb:nb + (cols // 128) * (K // 128)].reshape(cols // 128, K // 128), bs), g
+        assert np.array_equal(qb[:, o:o + K], bq), g
+        assert np.array_equal(sb[:, o // 128:(o + K) // 128], bs), g
 
 
 def test_swiglu_backward_quant(lib):
@@ -141,6 +142,40 @@ def test_grouped_scaled_gemm(lib, d, I, Kt, groups):
         if hi > lo:
             ref = O.scaled_gemm(aq[lo:hi], as_[lo:hi], *bs[gi])
             assert np.allclose(got[lo:hi], ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max()), gi
+
+
+@pytest.mark.parametrize("M,N,ranges", [(256, 512, [(0, 128), (128, 128), (128, 512), (512, 640)]),
+                                         (128, 256, [(0, 0), (0, 0)]),
+                                         (384, 768, [(0, 1024)])])
+def test_kgrouped_gemm(lib, M, N, ranges):
+    """c[g] = a[:, K_g] b[:, K_g]^T over each group's own K range (wgrad's
+    form), empty ranges giving zero, against the oracle's scaled GEMM."""
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    K = max(hi for _, hi in ranges)
+    rng = np.random.default_rng(M + N + K)
+    Kp = max(K, 128)
+    a = round_fp32(rng.standard_normal((M, Kp)) * np.exp2(rng.integers(-3, 3, (M, 1))))
+    b = round_fp32(rng.standard_normal((N, Kp)) * 0.05)
+    aq, as_ = O.quant_1x128(a)
+    bq, bs = O.quant_128x128(b)
+    kofs = np.array([lo for lo, _ in ranges] + [ranges[-1][1]], np.int32)
+    cu = lambda x, dt: torch.from_numpy(np.ascontiguousarray(x)).to(dt).cuda()
+    G = len(ranges)
+    c = torch.full((G, M, N), float("nan"), device="cuda")
+    ws = torch.empty(B.moe_kgrouped_gemm_fp8_workspace(), dtype=torch.uint8, device="cuda")
+    # K = 0 (every group empty) passes empty operands
+    B.moe_kgrouped_gemm_fp8(cu(aq[:, :K], torch.uint8), cu(as_[:, :K // 128], torch.float32),
+                            cu(bq[:, :K], torch.uint8), cu(bs[:, :K // 128], torch.float32),
+                            cu(kofs, torch.int32), c, ws)
+    torch.cuda.synchronize()
+    assert B.moe_get_error() == 0
+    got = c.cpu().double().numpy()
+    for g, (lo, hi) in enumerate(ranges):
+        if hi == lo:
+            assert np.array_equal(got[g], np.zeros((M, N))), g
+            continue
+        ref = O.scaled_gemm(aq[:, lo:hi], as_[:, lo // 128:hi // 128], bq[:, lo:hi], bs[:, lo // 128:hi // 128])
+        assert np.allclose(got[g], ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max()), g
 
 
 @pytest.mark.parametrize("cfg", [workloads.MoEConfig("bwd_small", T=150, d=512, N_r=4, K_r=2, I=256, seed=21),
