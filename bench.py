@@ -424,7 +424,8 @@ def backward_run(layer, u, e, b, b0, cfg, dev, peaks, steps=3):
     """The expert FFNs' FP8 backward on the same layer after one forward, with
     a seeded BF16 gradient of the expert outputs: dgrad (G and U recomputed,
     dH, SwiGLU backward, dX; 4 grouped GEMMs) and wgrad (three weight
-    gradients per expert) timed apart with CUDA events, `steps` each."""
+    gradients per expert, one K-grouped launch per weight) timed apart with
+    CUDA events, `steps` each."""
     import torch
 
     from fine_grained_fp8_sigmoid_b200 import binding as B
@@ -460,6 +461,7 @@ def backward_run(layer, u, e, b, b0, cfg, dev, peaks, steps=3):
     fl_dg = 2.0 * pairs * cfg.d * cfg.I * 5  # G, U recomputed, dH, and dX (K = 2I: twice)
     fl_wg = 2.0 * pairs * cfg.d * cfg.I * 3
     fp8 = 2.0 * peaks["bf16"]
+    grad_bytes = 4.0 * (cfg.N_r + 1) * 3 * cfg.d * cfg.I
     del bw, r, dy, xq, xs
     torch.cuda.empty_cache()
     return {"what": "expert FFN FP8 backward after one forward, BF16 dY of all routed and shared rows",
@@ -468,7 +470,11 @@ def backward_run(layer, u, e, b, b0, cfg, dev, peaks, steps=3):
                       "frac_of_fp8_burst": fl_dg / (dg_ms / 1e3) / 1e12 / fp8, "gemms": 4},
             "wgrad": {"ms": wg_ms, "tflops": fl_wg / (wg_ms / 1e3) / 1e12,
                       "frac_of_fp8_burst": fl_wg / (wg_ms / 1e3) / 1e12 / fp8,
-                      "gemms": 3 * (cfg.N_r + 1), "note": "one GEMM launch per expert and weight"}}
+                      # bound by writing the FP32 gradients of every expert
+                      "gradient_bytes": grad_bytes, "gbs": grad_bytes / (wg_ms / 1e3) / 1e9,
+                      "frac_of_hbm": grad_bytes / (wg_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                      "gemms": 3, "note": "one K-grouped GEMM launch per weight, every expert over its own tokens; "
+                                          "plus five transposed quantisations"}}
 
 
 def sub_workload(name, args, dev, world, local_rank, peaks):
