@@ -27,6 +27,7 @@ SIGNATURES = {
     "moe_quant_1x128": (_i, [_p, _i, _i, _p, _p, _p]),
     "moe_quant_128x128": (_i, [_p, _i, _i, _p, _p, _p]),
     "moe_route": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p]),
+    "moe_route_quant": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]),
     "moe_permute_workspace": (_z, [_i, _i]),
     "moe_permute": (_i, [_p, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p, _z, _p]),
     "moe_permute_noalloc": (_i, [_p, _i, _i, _i, _p, _p, _i, _p, _p, _p, _p, _p, _p, _p]),

@@ -80,6 +80,24 @@ def moe_route(u, e, b, K_r, topk_idx, gates, scores_in=None, scores_out=None, st
         _ptr(topk_idx), _ptr(gates), _stream(stream)))
 
 
+def moe_route_quant(u, e, b, K_r, topk_idx, gates, xq, xs, scores_out=None, stream=None):
+    """moe_route from u and e, and in the same kernel moe_quant_1x128 of u
+    into xq [T][d] (E4M3) and xs [T][d/128]."""
+    N_r = b.shape[0]
+    T, d = u.shape
+    _want(u, torch.bfloat16, (T, d), "u")
+    _want(e, torch.bfloat16, (N_r, d), "e")
+    _want(b, torch.float32, (N_r,), "b")
+    _want(topk_idx, torch.int32, (T, K_r), "topk_idx")
+    _want(gates, torch.float32, (T, K_r), "gates")
+    _want(xq, torch.uint8, (T, d), "xq")
+    _want(xs, torch.float32, (T, d // 128), "xs")
+    _opt(scores_out, torch.float32, (T, N_r), "scores_out")
+    check("moe_route_quant", _lib.load().moe_route_quant(
+        _ptr(u), _ptr(e), _ptr(b), T, d, N_r, K_r, _ptr(scores_out), _ptr(topk_idx), _ptr(gates),
+        _ptr(xq), _ptr(xs), _stream(stream)))
+
+
 def moe_permute_workspace(T, N_r):
     return int(_lib.load().moe_permute_workspace(T, N_r))
 

@@ -28,6 +28,17 @@
 // rank's shared memory alive until all ranks have read it.
 // Warp roles (384 threads): warp 0 TMA, warp 1 MMA + TMEM, warps 4-11
 // epilogue (TMEM lane quadrant w%4, column half (w-4)/4 while reading TMEM).
+//
+// Fused activation quantisation (xq non-null): the u tiles that stream
+// through shared memory for the logits are also the input of step 5 of the
+// layer, E4M3 in 1x128 tiles ("DeepSeek-V3 Teknik Raporu", Temel fikirler,
+// FP8 bullet). Two consecutive 64-channel K blocks hold one 1x128 tile per
+// token: epilogue thread (token r, half h) reads its token's 64 values of K
+// block 2p + h from the stage (otherwise idle during the K loop: the MMAs
+// are the logits' critical path), the two halves' max-abs meet through a
+// named barrier, and each half writes its 64 codes (half 0 the scale) with
+// the same arithmetic as moe_quant_1x128. A stage is refilled only after the
+// MMA commit and the four warps that read it have released it.
 #include <mutex>
 
 #include "host.cuh"
@@ -132,6 +143,7 @@ struct Smem {
   uint32_t tmem_base;
   int abort;
   float bias[NP];
+  float qamax[2][2][BM];      // fused quantisation: [pair parity][half][token] max-abs
 };
 
 static_assert(BM * PR * 4 <= STAGES * STAGE_BYTES, "parked logits fit the pipeline stages");
@@ -186,12 +198,36 @@ __device__ __forceinline__ void topk_insert_lex(float (&kk)[KMAX], int (&ii)[KMA
   }
 }
 
+// Named barrier over n threads that also ORs a predicate across them.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Eight bf16 of a 16-byte chunk as floats.
+__device__ __forceinline__ void bf16x8(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFF);
+    f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+  }
+}
+
 template <int KMAX>
 __global__ void __launch_bounds__(THREADS, 1)
     router_kernel(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_e,
                   const float* __restrict__ b, int T, int d, int N_r, int K, int S,
                   float* __restrict__ scores_out, int32_t* __restrict__ topk_idx,
-                  float* __restrict__ gates) {
+                  float* __restrict__ gates, uint8_t* __restrict__ xq, float* __restrict__ xs) {
   extern __shared__ uint8_t smem_raw[];
   // operand tiles need 1024-byte alignment for the 128-byte swizzle
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -210,7 +246,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+      // the MMA commit, and with the fused quantisation the four epilogue
+      // warps that read the stage's u rows
+      mbar_init(&sm.empty[s], xq != nullptr ? 1 + 4 : 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.tfull[i], 1);
@@ -293,9 +331,58 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
     bool ok = true;
     const int NG = g_hi - g_lo;
+    int qpar = 0;
     for (int grp = 0; grp < NG; ++grp) {
+      if (xq != nullptr) {
+        // quantise the 1x128 tiles of this partial group's K blocks
+        const int kb_a = kb_lo + grp * RK, kb_b = min(kb_a + RK, kb_hi);
+        for (int kb0 = kb_a; kb0 < kb_b; kb0 += 2) {
+          const int kb = kb0 + half;
+          const int st = (kb - kb_lo) % STAGES;
+          const bool okw = warp_wait(&sm.full[st], ((kb - kb_lo) / STAGES) & 1, abort);
+          const uint8_t* urow = tiles + st * STAGE_BYTES + r * 128;   // 128-byte swizzled row r
+          float amax = 0.0f;
+          if (okw) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              float f[8];
+              bf16x8(*reinterpret_cast<const uint4*>(urow + ((c ^ (r & 7)) << 4)), f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            }
+          }
+          sm.qamax[qpar][half][r] = amax;
+          if (named_bar_or(2, EPI_THREADS, !okw || *abort)) { ok = false; break; }
+          amax = fmaxf(amax, sm.qamax[qpar][half ^ 1][r]);
+          qpar ^= 1;
+          const float sc = tile_scale(amax);
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float f[8];
+            bf16x8(*reinterpret_cast<const uint4*>(urow + ((c ^ (r & 7)) << 4)), f);
+            w[2 * c] = e4m3x2(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc)) |
+                       (e4m3x2(__fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)) << 16);
+            w[2 * c + 1] = e4m3x2(__fdiv_rn(f[4], sc), __fdiv_rn(f[5], sc)) |
+                           (e4m3x2(__fdiv_rn(f[6], sc), __fdiv_rn(f[7], sc)) << 16);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.empty[st]);     // this warp is done with the stage
+          const int tok = tile * BM + r;
+          if (tok < T) {
+            uint4* dst = reinterpret_cast<uint4*>(xq + static_cast<size_t>(tok) * d + kb * BK);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            if (half == 0) xs[static_cast<size_t>(tok) * (d / 128) + kb0 / 2] = sc;
+          }
+        }
+        if (!ok) break;
+      }
       const int buf = grp & 1;
-      if (!warp_wait(&sm.tfull[buf], (grp >> 1) & 1, abort)) { ok = false; break; }
+      const bool okt = warp_wait(&sm.tfull[buf], (grp >> 1) & 1, abort);
+      // with the fused quantisation every epilogue warp must leave the loop
+      // together (its barriers count all of them)
+      if (xq != nullptr ? named_bar_or(2, EPI_THREADS, !okt) : !okt) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -450,9 +537,9 @@ __global__ void __launch_bounds__(128)
 }  // namespace route
 }  // namespace moe
 
-extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
-                         const float* scores_in, int T, int d, int N_r, int K_r,
-                         float* scores_out, int32_t* topk_idx, float* gates, void* stream) {
+static int route_launch(const uint16_t* u, const uint16_t* e, const float* b, const float* scores_in, int T, int d,
+                        int N_r, int K_r, float* scores_out, int32_t* topk_idx, float* gates, uint8_t* xq, float* xs,
+                        void* stream) {
   using namespace moe;
   using namespace moe::route;
   MOE_CHECK_ARG(T >= 0 && d >= 0 && N_r >= 1 && K_r >= 1);
@@ -520,8 +607,27 @@ extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
   while (S < max_cluster[dev][variant] && tiles * S * 2 <= di.sm_count && S * 2 <= NG_all) S *= 2;
   cfg.gridDim = dim3(tiles * S);
   attr[0].val.clusterDim.x = S;
-  if (int st = cuda_status(cudaLaunchKernelEx(&cfg, k, tm_u, tm_e, b, T, d, N_r, K_r, S, scores_out, topk_idx, gates),
+  if (int st = cuda_status(cudaLaunchKernelEx(&cfg, k, tm_u, tm_e, b, T, d, N_r, K_r, S, scores_out, topk_idx, gates,
+                                              xq, xs),
                            "router launch"))
     return st;
   return launch_status();
+}
+
+extern "C" int moe_route(const uint16_t* u, const uint16_t* e, const float* b, const float* scores_in, int T, int d,
+                         int N_r, int K_r, float* scores_out, int32_t* topk_idx, float* gates, void* stream) {
+  return route_launch(u, e, b, scores_in, T, d, N_r, K_r, scores_out, topk_idx, gates, nullptr, nullptr, stream);
+}
+
+extern "C" int moe_route_quant(const uint16_t* u, const uint16_t* e, const float* b, int T, int d, int N_r, int K_r,
+                               float* scores_out, int32_t* topk_idx, float* gates, uint8_t* xq, float* xs,
+                               void* stream) {
+  using namespace moe;
+  MOE_CHECK_ARG(T >= 0 && d >= 0);
+  MOE_CHECK_SUPPORTED(d % 128 == 0);
+  if (T > 0) {
+    MOE_CHECK_ARG(u && xq && xs);
+    MOE_CHECK_ARG(reinterpret_cast<uintptr_t>(xq) % 16 == 0);
+  }
+  return route_launch(u, e, b, nullptr, T, d, N_r, K_r, scores_out, topk_idx, gates, xq, xs, stream);
 }

@@ -132,6 +132,21 @@ MOE_API int moe_route(const uint16_t* u, const uint16_t* e, const float* b,
               void* stream);
 
 /*
+ * moe_route_quant: moe_route from u and e (no scores_in) and, in the same
+ * kernel, moe_quant_1x128 of u ("DeepSeek-V3 Teknik Raporu", Temel
+ * fikirler, FP8 bullet: activations in 1x128 tiles): the router's epilogue
+ * quantises the u tiles it streams for the logits, so u is read once for
+ * both steps.
+ *   xq, xs   [T][d] E4M3 and [T][d/128] FP32 (out): bit for bit what
+ *            moe_quant_1x128(u) writes
+ * Other arguments, outputs and limits as moe_route, and d a multiple of 128.
+ */
+MOE_API int moe_route_quant(const uint16_t* u, const uint16_t* e, const float* b,
+                    int T, int d, int N_r, int K_r, float* scores_out,
+                    int32_t* topk_idx, float* gates, uint8_t* xq, float* xs,
+                    void* stream);
+
+/*
  * moe_permute_workspace: bytes of scratch moe_permute needs for T tokens and
  * N_r experts (two int32 tables of ceil(T/256) x N_r).
  */

@@ -83,6 +83,8 @@ def test_host_side_argument_checks(lib):
                                     N, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_grouped_gemm_fp8(N, N, N, 8, 2, N, N, 4, N, N, N, N, N, N, 256, 100,
                                     N, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
+    # fused router + quantisation: d not a multiple of 128
+    assert lib.moe_route_quant(N, N, N, 4, 192, 8, 2, N, N, N, N, N, s) == _lib.MOE_ERR_UNSUPPORTED
     # K-grouped GEMM: M not a multiple of 128, N not a multiple of 256, G = 0
     assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 4, 100, 256, 128, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED
     assert lib.moe_kgrouped_gemm_fp8(N, N, N, N, N, 4, 128, 384, 128, N, N, 0, s) == _lib.MOE_ERR_UNSUPPORTED

@@ -125,6 +125,44 @@ def test_router_tensor_cores(lib, name, T, K):
     assert np.allclose(gates.cpu().double().numpy(), rg, rtol=1e-4, atol=1e-6)
 
 
+@pytest.mark.parametrize("name,T,K", [("tiny", None, None), ("mid", 1000, None), ("prefill", 1500, None),
+                                      ("prefill", 1, None), ("decode", None, None), ("mid", 5000, 16)])
+def test_route_quant_fused(lib, name, T, K):
+    """moe_route_quant: the router's own outputs equal moe_route's bit for
+    bit, and its xq/xs equal the oracle's 1x128 quantisation of u bit for bit
+    (incl. a ragged last token tile, one token, and the cluster-split decode
+    launch where each rank quantises its share of the channels)."""
+    import dataclasses
+    from fine_grained_fp8_sigmoid_b200 import binding as B
+    cfg = workloads.CONFIGS[name]
+    if T is not None:
+        cfg = cfg.with_tokens(T)
+    if K is not None:
+        cfg = dataclasses.replace(cfg, K_r=K)
+    u, e, b = workloads.activations(cfg), workloads.centroids(cfg), workloads.bias(cfg)
+    if cfg.T >= 4 and cfg.d >= 256:   # special tiles: zero, -0, bf16 subnormal, +-448
+        u = u.clone()
+        u[0, :128] = 0.0
+        u[1, 128:256] = -0.0
+        u[2, :128] = (torch.randn(128, generator=torch.Generator().manual_seed(5)) * 2.0 ** -130).to(u.dtype)
+        u[3, :128] = 448.0
+    ud, ed, bd = u.cuda(), e.cuda(), b.cuda()
+    out = lambda: (torch.empty(cfg.T, cfg.K_r, dtype=torch.int32, device="cuda"),
+                   torch.empty(cfg.T, cfg.K_r, dtype=torch.float32, device="cuda"))
+    idx0, g0 = out()
+    idx1, g1 = out()
+    xq = torch.full((cfg.T, cfg.d), 0x55, dtype=torch.uint8, device="cuda")
+    xs = torch.full((cfg.T, cfg.d // 128), -1.0, device="cuda")
+    B.moe_route(ud, ed, bd, cfg.K_r, idx0, g0)
+    B.moe_route_quant(ud, ed, bd, cfg.K_r, idx1, g1, xq, xs)
+    torch.cuda.synchronize()
+    assert B.moe_get_error() == 0
+    assert torch.equal(idx0, idx1) and torch.equal(g0, g1)
+    rq, rs = O.quant_1x128(u.double().numpy())
+    assert np.array_equal(xq.cpu().numpy(), rq)
+    assert np.array_equal(xs.cpu().double().numpy(), rs)
+
+
 def _tied_centroids(cfg, mode):
     """Centroids with exactly repeated rows, so that logits (and with equal
     bias, keys) tie bit for bit. mode "pairs": a few expert pairs share a

@@ -36,9 +36,9 @@ def _threads():
     return max(2, min(32, os.cpu_count() or 8))
 
 
-def _build(cfg, weights_on="cuda", gather=None):
+def _build(cfg, weights_on="cuda", gather=None, fuse_quant=False):
     from fine_grained_fp8_sigmoid_b200 import MoELayerFP8
-    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, gather=gather)
+    layer = MoELayerFP8(cfg.T, cfg.d, cfg.N_r, cfg.K_r, cfg.I, gather=gather, fuse_quant=fuse_quant)
     for slot in range(cfg.N_r + 1):
         w = workloads.expert_weights(cfg, slot, device=weights_on)
         layer.load_expert(slot, *[x.cuda() for x in w])
@@ -210,6 +210,26 @@ def test_layer_gather_fused_equals_materialised(lib, name):
         bb = b.clone()
         outs.append((layer.forward(u, e, bb).clone(), layer.y_perm.clone(), bb))
         torch.cuda.synchronize()
+    for a_, b_ in zip(*outs):
+        assert torch.equal(a_, b_)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_layer_fused_quantisation_equals_separate(lib, name):
+    """The layer with the activation quantisation fused into the router and
+    with moe_quant_1x128 apart give the same xq, xs and h', bit for bit."""
+    cfg = workloads.CONFIGS[name]
+    u = workloads.activations(cfg, device="cuda")
+    e = workloads.centroids(cfg, device="cuda")
+    b = workloads.bias(cfg, device="cuda")
+    outs = []
+    for fuse in (True, False):
+        layer = _build(cfg, "cuda", fuse_quant=fuse)
+        bb = b.clone()
+        out = layer.forward(u, e, bb).clone()
+        torch.cuda.synchronize()
+        outs.append((out, layer.xq.clone(), layer.xs.clone(), bb))
+        assert layer.launches_per_step() == (9 if fuse else 10) - (1 if layer.gather else 0)
     for a_, b_ in zip(*outs):
         assert torch.equal(a_, b_)
 
