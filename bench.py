@@ -106,12 +106,12 @@ def gemm_algorithmic_bytes(cfg, touched_routed):
     """Bytes one moe_grouped_gemm_fp8 call must move at least: the weights of
     the touched routed experts and the shared one, read once; the permuted
     and shared activations with their scales; the intermediate H written and
-    read back; the FP32 outputs written."""
+    read back; the bf16 outputs written."""
     per_expert = 3 * cfg.d * cfg.I + 3 * (cfg.d // 128) * (cfg.I // 128) * 4
     rows = cfg.T * cfg.K_r + cfg.T
     acts = rows * (cfg.d + cfg.d // 128 * 4)
     inter = 2 * rows * (cfg.I + cfg.I // 128 * 4)
-    outs = rows * cfg.d * 4
+    outs = rows * cfg.d * 2
     return (touched_routed + 1) * per_expert + acts + inter + outs
 
 

@@ -51,6 +51,7 @@ SIGNATURES = {
     "moe_quant_128x128_t": (_i, [_p, _p, _i, _i, _p, _p, _i, _i, _p, _p, _p]),
     "moe_transpose": (_i, [_p, _i, _i, _i, _i, _p, _i, _i, _p]),
     "moe_combine": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
+    "moe_combine_fp32": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _p, _p]),
     "moe_bias_update": (_i, [_p, _p, _i, _i, _i, _f, _p, _p]),
     "moe_debug_wait_timeout": (_i, [_i, _p]),
 }

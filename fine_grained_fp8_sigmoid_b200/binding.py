@@ -172,8 +172,8 @@ def moe_grouped_gemm_fp8(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w_down
     _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
     _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
     _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
-    _want(y_perm, torch.float32, (P, d), "y_perm")
-    _want(y_shared, torch.float32, (T, d), "y_shared")
+    _want(y_perm, torch.bfloat16, (P, d), "y_perm")
+    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
     if T and P != T * K_r:
         raise ValueError("xq_perm rows must be T * K_r")
     check("moe_grouped_gemm_fp8", _lib.load().moe_grouped_gemm_fp8(
@@ -201,8 +201,8 @@ def moe_grouped_gemm_fp8_gather(sorted_token, offsets, xq, xs, w_gate, w_up, w_d
     _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
     _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
     _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
-    _want(y_perm, torch.float32, (P, d), "y_perm")
-    _want(y_shared, torch.float32, (T, d), "y_shared")
+    _want(y_perm, torch.bfloat16, (P, d), "y_perm")
+    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
     if T and P != T * K_r:
         raise ValueError("sorted_token must hold T * K_r rows")
     check("moe_grouped_gemm_fp8_gather", _lib.load().moe_grouped_gemm_fp8_gather(
@@ -235,8 +235,8 @@ def moe_grouped_gemm_fp8_rows(xq_perm, xs_perm, offsets, xq, xs, w_gate, w_up, w
     _want(s_gate, torch.float32, (G, I // 128, d // 128), "s_gate")
     _want(s_up, torch.float32, (G, I // 128, d // 128), "s_up")
     _want(s_down, torch.float32, (G, d // 128, I // 128), "s_down")
-    _want(y_perm, torch.float32, (P, d), "y_perm")
-    _want(y_shared, torch.float32, (T, d), "y_shared")
+    _want(y_perm, torch.bfloat16, (P, d), "y_perm")
+    _want(y_shared, torch.bfloat16, (T, d), "y_shared")
     check("moe_grouped_gemm_fp8_rows", _lib.load().moe_grouped_gemm_fp8_rows(
         _ptr(xq_perm), _ptr(xs_perm), _ptr(offsets), N, P, _ptr(xq), _ptr(xs), T,
         _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(s_gate), _ptr(s_up), _ptr(s_down),
@@ -379,15 +379,20 @@ def moe_transpose(src, dst, dst_col=0, stream=None):
 
 
 def moe_combine(u, y_perm, y_shared, inv, gates, out, stream=None):
+    """h' from bf16 expert rows (moe_combine), or FP32 rows (moe_combine_fp32)."""
     T, d = u.shape
     K_r = inv.shape[1]
+    dt = y_perm.dtype
+    if dt not in (torch.bfloat16, torch.float32):
+        raise ValueError("y_perm must be bf16 or FP32")
     _want(u, torch.bfloat16, (T, d), "u")
-    _want(y_perm, torch.float32, (T * K_r, d), "y_perm")
-    _want(y_shared, torch.float32, (T, d), "y_shared")
+    _want(y_perm, dt, (T * K_r, d), "y_perm")
+    _want(y_shared, dt, (T, d), "y_shared")
     _want(inv, torch.int32, (T, K_r), "inv")
     _want(gates, torch.float32, (T, K_r), "gates")
     _want(out, torch.bfloat16, (T, d), "out")
-    check("moe_combine", _lib.load().moe_combine(
+    fn = _lib.load().moe_combine if dt == torch.bfloat16 else _lib.load().moe_combine_fp32
+    check("moe_combine", fn(
         _ptr(u), _ptr(y_perm), _ptr(y_shared), _ptr(inv), _ptr(gates), T, K_r, d, _ptr(out),
         _stream(stream)))
 

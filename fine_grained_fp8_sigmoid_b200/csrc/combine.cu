@@ -6,15 +6,53 @@
 namespace moe {
 
 // One block per token; each thread handles 8 consecutive channels (16 bytes
-// of bf16) per step. FP32 sum in the fixed order: u, shared, k = 0..K-1.
+// of bf16 from u, the shared row and every routed row) per step, all the
+// step's loads issued before the sums. FP32 sum in the fixed order: u,
+// shared, k = 0..K-1.
+constexpr int COMBINE_KMAX = 16;
+
+__device__ __forceinline__ void bf16x8_to_float(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16_bits_to_float(w[i] & 0xFFFF);
+    f[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+  }
+}
+
+// Eight values of a row as floats: bf16 (one 16-byte load) or FP32 (two).
+template <typename Y>
+struct Row8;
+template <>
+struct Row8<uint16_t> {
+  uint4 v;
+  __device__ __forceinline__ void load(const uint16_t* p) { v = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void zero() { v = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void get(float (&f)[8]) const { bf16x8_to_float(v, f); }
+};
+template <>
+struct Row8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p + 4));
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void get(float (&f)[8]) const {
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+};
+
+template <typename Y>
 __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict__ u,
-                                                      const float* __restrict__ y_perm,
-                                                      const float* __restrict__ y_shared,
+                                                      const Y* __restrict__ y_perm,
+                                                      const Y* __restrict__ y_shared,
                                                       const int32_t* __restrict__ inv,
                                                       const float* __restrict__ gates, int K,
                                                       int d, int P, uint16_t* out) {
-  __shared__ int s_row[16];
-  __shared__ float s_g[16];
+  __shared__ int s_row[COMBINE_KMAX];
+  __shared__ float s_g[COMBINE_KMAX];
   const int t = blockIdx.x;
   if (threadIdx.x < K) {
     int r = inv[static_cast<size_t>(t) * K + threadIdx.x];
@@ -29,26 +67,26 @@ __global__ void __launch_bounds__(128) combine_kernel(const uint16_t* __restrict
   const size_t base = static_cast<size_t>(t) * d;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     const uint4 a = *reinterpret_cast<const uint4*>(u + base + c);
-    const float4 sh0 = __ldg(reinterpret_cast<const float4*>(y_shared + base + c));
-    const float4 sh1 = __ldg(reinterpret_cast<const float4*>(y_shared + base + c + 4));
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-    const float sv[8] = {sh0.x, sh0.y, sh0.z, sh0.w, sh1.x, sh1.y, sh1.z, sh1.w};
-    float acc[8];
+    Row8<Y> sh;
+    sh.load(y_shared + base + c);
+    Row8<Y> yv[COMBINE_KMAX];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[2 * i] = bf16_bits_to_float(aw[i] & 0xFFFF) + sv[2 * i];
-      acc[2 * i + 1] = bf16_bits_to_float(aw[i] >> 16) + sv[2 * i + 1];
+    for (int k = 0; k < COMBINE_KMAX; ++k) {
+      yv[k].zero();
+      if (k < K && s_row[k] >= 0) yv[k].load(y_perm + static_cast<size_t>(s_row[k]) * d + c);
     }
-    for (int k = 0; k < K; ++k) {
-      const int r = s_row[k];
-      if (r < 0) continue;
-      const float g = s_g[k];
-      const float* yr = y_perm + static_cast<size_t>(r) * d + c;
-      const float4 y0 = __ldg(reinterpret_cast<const float4*>(yr));
-      const float4 y1 = __ldg(reinterpret_cast<const float4*>(yr + 4));
-      const float yv[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+    float acc[8], f[8];
+    bf16x8_to_float(a, acc);
+    sh.get(f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, yv[i], acc[i]);
+    for (int i = 0; i < 8; ++i) acc[i] += f[i];
+#pragma unroll
+    for (int k = 0; k < COMBINE_KMAX; ++k) {
+      if (k >= K || s_row[k] < 0) continue;
+      const float g = s_g[k];
+      yv[k].get(f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(g, f[i], acc[i]);
     }
     uint4 o;
     o.x = float_to_bf16_bits(acc[0]) | (static_cast<uint32_t>(float_to_bf16_bits(acc[1])) << 16);
@@ -104,9 +142,9 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
 
 }  // namespace moe
 
-extern "C" int moe_combine(const uint16_t* u, const float* y_perm, const float* y_shared,
-                           const int32_t* inv, const float* gates, int T, int K_r, int d,
-                           uint16_t* out, void* stream) {
+template <typename Y>
+static int combine(const uint16_t* u, const Y* y_perm, const Y* y_shared, const int32_t* inv, const float* gates,
+                   int T, int K_r, int d, uint16_t* out, void* stream) {
   using namespace moe;
   MOE_CHECK_ARG(T >= 0 && K_r >= 1 && d >= 0);
   MOE_CHECK_SUPPORTED(K_r <= 16 && d % 8 == 0);
@@ -117,8 +155,20 @@ extern "C" int moe_combine(const uint16_t* u, const float* y_perm, const float* 
   MOE_CHECK_SUPPORTED(static_cast<long long>(T) * K_r < (1LL << 31));
   DeviceInfo di;
   if (int st = device_info(&di)) return st;
-  combine_kernel<<<T, 128, 0, as_stream(stream)>>>(u, y_perm, y_shared, inv, gates, K_r, d, T * K_r, out);
+  combine_kernel<Y><<<T, 128, 0, as_stream(stream)>>>(u, y_perm, y_shared, inv, gates, K_r, d, T * K_r, out);
   return launch_status();
+}
+
+extern "C" int moe_combine(const uint16_t* u, const uint16_t* y_perm, const uint16_t* y_shared,
+                           const int32_t* inv, const float* gates, int T, int K_r, int d,
+                           uint16_t* out, void* stream) {
+  return combine(u, y_perm, y_shared, inv, gates, T, K_r, d, out, stream);
+}
+
+extern "C" int moe_combine_fp32(const uint16_t* u, const float* y_perm, const float* y_shared,
+                                const int32_t* inv, const float* gates, int T, int K_r, int d,
+                                uint16_t* out, void* stream) {
+  return combine(u, y_perm, y_shared, inv, gates, T, K_r, d, out, stream);
 }
 
 extern "C" int moe_bias_update(float* b, const int32_t* counts, int N_r, int T, int K_r, float gamma,

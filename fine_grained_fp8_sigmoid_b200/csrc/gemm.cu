@@ -121,8 +121,9 @@ struct Args {
   const float* s_down;
   uint8_t* H;
   float* Hs;
-  float* y_perm;
-  float* y_shared;
+  void* y_perm;              // phase-2 output rows: FP32, or bf16 when y_bf16
+  void* y_shared;
+  int y_bf16;
   int* tile_counter;         // zeroed before the launch; tiles past the first wave are claimed from it
   const int32_t* sorted_token;  // non-null: routed rows are read from xq/xs at these tokens (no xq_perm)
   // K-grouped (phase 2 only): N_r + 1 groups share A's T rows and B's rows;
@@ -231,6 +232,11 @@ __device__ __forceinline__ Tile decode_tile(const S& sm, const Args& a, int t, i
 // silu(x) = x / (1 + e^-x) with the fast exponential and division: branch-free
 // (x -> -inf gives e^-x = inf and x / inf = -0, the limit).
 __device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+
+// Two floats rounded to bf16 (round to nearest even), packed low | high << 16.
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  return static_cast<uint32_t>(float_to_bf16_bits(lo)) | (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
+}
 
 // 2-D tiled store of one box from shared memory (bulk async group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int x, int y) {
@@ -420,13 +426,21 @@ __device__ __forceinline__ bool narrow_tile(S& sm, const Args& a, const Tile tl,
     }
   } else {
     // output channel n*256 + half*128 + c of each token: a warp writes 32
-    // consecutive channels (128 bytes) of one token at a time
-    float* y = (tl.shared ? a.y_shared + static_cast<size_t>(r0 - a.P) * a.d
-                          : a.y_perm + static_cast<size_t>(r0) * a.d) +
-               (tl.n * BN + x.half * 128 + c);
+    // consecutive channels of one token at a time
+    const size_t at = (tl.shared ? static_cast<size_t>(r0 - a.P) : static_cast<size_t>(r0)) * a.d +
+                      (tl.n * BN + x.half * 128 + c);
+    void* ybase = tl.shared ? a.y_shared : a.y_perm;
+    if (a.y_bf16) {
+      uint16_t* y = static_cast<uint16_t*>(ybase) + at;
 #pragma unroll
-    for (int j = 0; j < NV; ++j)
-      if (j < tl.mrows) y[static_cast<size_t>(j) * a.d] = acc[j];
+      for (int j = 0; j < NV; ++j)
+        if (j < tl.mrows) y[static_cast<size_t>(j) * a.d] = float_to_bf16_bits(acc[j]);
+    } else {
+      float* y = static_cast<float*>(ybase) + at;
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        if (j < tl.mrows) y[static_cast<size_t>(j) * a.d] = acc[j];
+    }
   }
   return true;
 }
@@ -844,7 +858,45 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row_first = tl.m * BM + q * 32;             // within the group
         const int nvalid = min(Y_BOX, tl.rows - row_first);
         const int col0 = tl.n * BN + half * 128;
-        if (nvalid == Y_BOX) {
+        const size_t yrow_at = tl.shared ? static_cast<size_t>(rr) : static_cast<size_t>(tl.orow0 + rr);
+        if (a.y_bf16 && nvalid == Y_BOX) {
+          // bf16 rows (the layer's expert outputs): two 32 x 64 boxes per
+          // warp, each lane's 64 values of a box rounded to bf16 and packed
+          // into the row's eight 16-byte chunks (swizzled as the FP32 boxes)
+          const CUtensorMap* ym = tl.shared ? &tm_ys : &tm_y;
+          const int ytop = tl.shared ? row_first : tl.orow0 + row_first;
+          uint8_t* wstage = staging + ew * 2 * Y_BOX_BYTES;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint8_t* box = wstage + c * Y_BOX_BYTES;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float* v = &acc[c * 64 + 8 * i];
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((i ^ (lane & 7)) * 16)) =
+                  make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]),
+                             bf16x2_bits(v[6], v[7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(ym, box, col0 + c * 64, ytop);
+              bulk_commit();
+            }
+          }
+        } else if (a.y_bf16) {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(
+                static_cast<uint16_t*>(tl.shared ? a.y_shared : a.y_perm) + yrow_at * a.d + col0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float* v = &acc[8 * i];
+              dst[i] = make_uint4(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]), bf16x2_bits(v[4], v[5]),
+                                  bf16x2_bits(v[6], v[7]));
+            }
+          }
+        } else if (nvalid == Y_BOX) {
           const CUtensorMap* ym = tl.shared ? &tm_ys : &tm_y;
           const int ytop = tl.shared ? row_first : tl.orow0 + row_first;
           uint8_t* wstage = staging + ew * 2 * Y_BOX_BYTES;
@@ -866,8 +918,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         } else if (valid) {
-          float* yrow = tl.shared ? a.y_shared + static_cast<size_t>(rr) * a.d
-                                  : a.y_perm + static_cast<size_t>(tl.orow0 + rr) * a.d;
+          float* yrow = static_cast<float*>(tl.shared ? a.y_shared : a.y_perm) + yrow_at * a.d;
           float4* dst = reinterpret_cast<float4*>(yrow + col0);
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -889,6 +940,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // 2-D row-major FP32 tensor stored in 32 x 32 boxes with the 128-byte swizzle.
+// 2-D row-major bf16 tensor stored in 32 x 64 boxes (128-byte rows) with the
+// 128-byte swizzle.
+inline int make_tmap_ybf(CUtensorMap* m, const uint16_t* base, uint64_t rows, uint64_t cols) {
+  return make_tmap_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, Y_BOX, 2 * Y_BOX);
+}
+
 inline int make_tmap_y(CUtensorMap* m, const float* base, uint64_t rows, uint64_t cols) {
   return make_tmap_2d(m, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols, Y_BOX, Y_BOX);
 }
@@ -932,7 +989,7 @@ extern "C" int moe_grouped_gemm_fp8_launches(int d, int I) {
 static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int32_t* sorted_token,
                         const int32_t* offsets, int N_r, long long P, const uint8_t* xq, const float* xs, int T,
                         const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down, const float* s_gate,
-                        const float* s_up, const float* s_down, int d, int I, float* y_perm, float* y_shared,
+                        const float* s_up, const float* s_down, int d, int I, uint16_t* y_perm, uint16_t* y_shared,
                         void* workspace, size_t ws_bytes, void* stream) {
   using namespace moe;
   using namespace moe::gg;
@@ -972,9 +1029,9 @@ static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int3
   if (int st = make_tmap_2d(&tmWu, w_up, U8, 1, static_cast<uint64_t>(N_r + 1) * I, d, 128, BK)) return st;
   if (int st = make_tmap_2d(&tmH, H, U8, 1, rowsH, I, BM, BK)) return st;
   if (int st = make_tmap_2d(&tmWd, w_down, U8, 1, static_cast<uint64_t>(N_r + 1) * d, I, BN, BK)) return st;
-  if (int st = make_tmap_y(&tmYs, y_shared, T, d)) return st;
+  if (int st = make_tmap_ybf(&tmYs, y_shared, T, d)) return st;
   if (P > 0) {
-    if (int st = make_tmap_y(&tmY, y_perm, P, d)) return st;
+    if (int st = make_tmap_ybf(&tmY, y_perm, P, d)) return st;
   } else {
     tmY = tmYs;
   }
@@ -1002,6 +1059,7 @@ static int grouped_gemm(const uint8_t* xq_perm, const float* xs_perm, const int3
   args.Hs = Hs;
   args.y_perm = y_perm;
   args.y_shared = y_shared;
+  args.y_bf16 = 1;
   args.narrow_max = narrow ? NMAX : 0;
   args.sorted_token = sorted_token;
   int* counters = reinterpret_cast<int*>(H + counters_offset(static_cast<size_t>(rowsH), I));
@@ -1036,7 +1094,7 @@ extern "C" int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm
                                     int N_r, int K_r, const uint8_t* xq, const float* xs, int T,
                                     const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
                                     const float* s_gate, const float* s_up, const float* s_down, int d,
-                                    int I, float* y_perm, float* y_shared, void* workspace,
+                                    int I, uint16_t* y_perm, uint16_t* y_shared, void* workspace,
                                     size_t ws_bytes, void* stream) {
   if (K_r < 1) return MOE_ERR_INVALID_ARG;
   return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_r, static_cast<long long>(T) * K_r, xq, xs, T, w_gate,
@@ -1047,7 +1105,7 @@ extern "C" int moe_grouped_gemm_fp8_rows(const uint8_t* xq_perm, const float* xs
                                          int N_groups, int P, const uint8_t* xq, const float* xs, int T,
                                          const uint8_t* w_gate, const uint8_t* w_up, const uint8_t* w_down,
                                          const float* s_gate, const float* s_up, const float* s_down, int d, int I,
-                                         float* y_perm, float* y_shared, void* workspace, size_t ws_bytes,
+                                         uint16_t* y_perm, uint16_t* y_shared, void* workspace, size_t ws_bytes,
                                          void* stream) {
   if (P < 0) return MOE_ERR_INVALID_ARG;
   return grouped_gemm(xq_perm, xs_perm, nullptr, offsets, N_groups, P, xq, xs, T, w_gate, w_up, w_down, s_gate, s_up,
@@ -1057,8 +1115,8 @@ extern "C" int moe_grouped_gemm_fp8_rows(const uint8_t* xq_perm, const float* xs
 extern "C" int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token, const int32_t* offsets, int N_r, int K_r,
                                            const uint8_t* xq, const float* xs, int T, const uint8_t* w_gate,
                                            const uint8_t* w_up, const uint8_t* w_down, const float* s_gate,
-                                           const float* s_up, const float* s_down, int d, int I, float* y_perm,
-                                           float* y_shared, void* workspace, size_t ws_bytes, void* stream) {
+                                           const float* s_up, const float* s_down, int d, int I, uint16_t* y_perm,
+                                           uint16_t* y_shared, void* workspace, size_t ws_bytes, void* stream) {
   // a null sorted_token falls to the materialised-rows check (INVALID_ARG)
   if (K_r < 1) return MOE_ERR_INVALID_ARG;
   return grouped_gemm(nullptr, nullptr, sorted_token, offsets, N_r, static_cast<long long>(T) * K_r, xq, xs, T,

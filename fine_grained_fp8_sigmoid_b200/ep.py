@@ -88,7 +88,7 @@ class GpuOps:
 
     def experts(self, xq_perm, xs_perm, offsets, xq, xs):
         P, T = xq_perm.shape[0], xq.shape[0]
-        y_perm, y_sh = self._empty(P, self.d, dtype=torch.float32), self._empty(T, self.d, dtype=torch.float32)
+        y_perm, y_sh = self._empty(P, self.d, dtype=torch.bfloat16), self._empty(T, self.d, dtype=torch.bfloat16)
         ws = self._empty(max(B.moe_grouped_gemm_fp8_rows_workspace(P, T, self.d, self.I), 256), dtype=torch.uint8)
         B.moe_grouped_gemm_fp8_rows(xq_perm, xs_perm, offsets, xq, xs, self.w_gate, self.w_up, self.w_down,
                                     self.s_gate, self.s_up, self.s_down, y_perm, y_sh, ws)

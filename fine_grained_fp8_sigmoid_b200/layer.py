@@ -60,8 +60,8 @@ class MoELayerFP8:
         self.inv = torch.empty(T, K_r, dtype=i32, **dev)
         self.xq_perm = None if gather else torch.empty(P, d, dtype=u8, **dev)
         self.xs_perm = None if gather else torch.empty(P, d // 128, dtype=f32, **dev)
-        self.y_perm = torch.empty(P, d, dtype=f32, **dev)
-        self.y_shared = torch.empty(T, d, dtype=f32, **dev)
+        self.y_perm = torch.empty(P, d, dtype=bf, **dev)
+        self.y_shared = torch.empty(T, d, dtype=bf, **dev)
         self.out = torch.empty(T, d, dtype=bf, **dev)
         self.max_over_mean = torch.zeros(1, dtype=f32, **dev)
         self.ws_perm = torch.empty(max(B.moe_permute_workspace(T, N_r), 16), dtype=u8, **dev)

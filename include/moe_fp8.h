@@ -229,7 +229,7 @@ MOE_API int moe_grouped_gemm_fp8_launches(int d, int I);
  * shared expert (slot N_r, all T rows of xq):
  *   G = X W_gate^T, U = X W_up^T      (FP8 x FP8 -> FP32)
  *   A = silu(G) * U,  H = quant_1x128(A)
- *   Y = H W_down^T, stored in FP32
+ *   Y = H W_down^T, summed in FP32 and stored rounded to bf16
  * Each product is sum over 128-wide K blocks kb of
  *   s_X[m,kb] * s_W[n/128,kb] * (X_kb . W_kb),
  * the block partial coming from the tensor cores and the scaling and the sum
@@ -239,14 +239,8 @@ MOE_API int moe_grouped_gemm_fp8_launches(int d, int I);
  *   xq, xs            [T][d], [T][d/128]: the shared expert's input
  *   w_gate, w_up      [N_r+1][I][d] E4M3;  s_gate, s_up  [N_r+1][I/128][d/128]
  *   w_down            [N_r+1][d][I] E4M3;  s_down        [N_r+1][d/128][I/128]
- *   y_perm            [P][d] FP32 (out)    y_shared [T][d] FP32 (out)
- *                     FP32, not bf16: h' is rounded to bf16 once, in
- *                     moe_combine. Rounding the expert outputs to bf16 as
- *                     well puts outputs near a bf16 midpoint one ulp apart
- *                     from the FP64 reference, which breaks the output
- *                     tolerance where h' cancels to about zero; the cost is
- *                     twice the output bytes (prefill: 2.11 GB written
- *                     instead of 1.06 GB, and the same read by moe_combine).
+ *   y_perm            [P][d] bf16 (out)    y_shared [T][d] bf16 (out)
+ *                     each element the FP32 result rounded to nearest even
  *   workspace         moe_grouped_gemm_fp8_workspace(T, K_r, d, I) bytes
  * Limits: d a multiple of 256, I a multiple of 128, N_r <= 1024.
  */
@@ -256,7 +250,7 @@ MOE_API int moe_grouped_gemm_fp8(const uint8_t* xq_perm, const float* xs_perm,
                          const uint8_t* w_gate, const uint8_t* w_up,
                          const uint8_t* w_down, const float* s_gate,
                          const float* s_up, const float* s_down, int d, int I,
-                         float* y_perm, float* y_shared,
+                         uint16_t* y_perm, uint16_t* y_shared,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
@@ -276,7 +270,7 @@ MOE_API int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token,
                          const uint8_t* w_gate, const uint8_t* w_up,
                          const uint8_t* w_down, const float* s_gate,
                          const float* s_up, const float* s_down, int d, int I,
-                         float* y_perm, float* y_shared,
+                         uint16_t* y_perm, uint16_t* y_shared,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
@@ -297,7 +291,7 @@ MOE_API int moe_grouped_gemm_fp8_rows(const uint8_t* xq_perm, const float* xs_pe
                          const uint8_t* w_gate, const uint8_t* w_up,
                          const uint8_t* w_down, const float* s_gate,
                          const float* s_up, const float* s_down, int d, int I,
-                         float* y_perm, float* y_shared,
+                         uint16_t* y_perm, uint16_t* y_shared,
                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
@@ -427,14 +421,23 @@ MOE_API int moe_transpose(const void* src, int elem_bytes, int batch, int rows, 
  * moe_combine: h'_t = bf16(u_t + y_shared_t + sum_k g_{t,k} y_perm[inv[t][k]])
  * ("DeepSeek-V3 Teknik Raporu", Yöntem 2, the h'_t equation). The sum is FP32
  * in the fixed order u, shared, k = 0..K_r-1.
- *   u [T][d] bf16;  y_shared [T][d] FP32;  y_perm [T*K_r][d] FP32;  inv, gates [T][K_r]
+ *   u [T][d] bf16;  y_shared [T][d] bf16;  y_perm [T*K_r][d] bf16;  inv, gates [T][K_r]
  *   out [T][d] bf16 (may alias u)
  * d must be a multiple of 8.
  */
-MOE_API int moe_combine(const uint16_t* u, const float* y_perm,
-                const float* y_shared, const int32_t* inv,
+MOE_API int moe_combine(const uint16_t* u, const uint16_t* y_perm,
+                const uint16_t* y_shared, const int32_t* inv,
                 const float* gates, int T, int K_r, int d, uint16_t* out,
                 void* stream);
+
+/*
+ * moe_combine_fp32: moe_combine with FP32 rows y_perm, y_shared (the
+ * backward sums the FP32 input gradients of a token's rows with it, gates 1).
+ */
+MOE_API int moe_combine_fp32(const uint16_t* u, const float* y_perm,
+                     const float* y_shared, const int32_t* inv,
+                     const float* gates, int T, int K_r, int d, uint16_t* out,
+                     void* stream);
 
 /*
  * moe_bias_update: auxiliary-loss-free balancing ("DeepSeek-V3 Teknik

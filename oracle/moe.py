@@ -182,8 +182,8 @@ def expert_ffn_parts(xq, xs, w: dict) -> dict:
 
     a = silu(X W_gate^T) * (X W_up^T); a is rounded to FP32 (the precision
     the kernel holds it in) and requantised per 1x128 tile along I to
-    (hq, hs); then Y = H W_down^T, kept in float64 (the exact target of the
-    kernel's FP32 output).
+    (hq, hs); then Y = H W_down^T, kept in float64 here (the exact value
+    that the layer's bf16 expert output rounds; moe_forward rounds it).
     Returns dict(G, U, a32 [m, I], hq uint8 [m, I], hs [m, I/128], y [m, d]).
     """
     G = scaled_gemm(xq, xs, w["gate_q"], w["gate_s"])
@@ -374,13 +374,18 @@ def moe_forward(u, e, b, K: int, weights, tokens=None, select=None, map_fn=map) 
                 if "hq" in routed else None)
     h_shared = dequant_1x128(shared["hq"], shared["hs"])
 
-    acc = u[sample] + y_shared
+    # the expert outputs cross to the combine as bf16 (reading: the layer's
+    # activations are bf16 on both sides of the FFNs, [TR] Yöntem 2 h'_t
+    # equation), and h' is rounded to bf16 once more after the sum
+    y_routed_bf16, y_shared_bf16 = round_bf16(y_routed), round_bf16(y_shared)
+    acc = u[sample] + y_shared_bf16
     for k in range(K):
-        acc = acc + gates[sample, k:k + 1] * y_routed[:, k]
+        acc = acc + gates[sample, k:k + 1] * y_routed_bf16[:, k]
     out = round_bf16(acc)
     return dict(scores=s, scores32=s32, topk_idx=idx, gates=gates,
                 counts=counts, offsets=offsets, sorted_token=sorted_token,
                 inv=inv, bias_new=b_new, max_over_mean=ratio, tokens=sample,
                 xq=xq, xs=xs, y_routed=y_routed, h_routed=h_routed,
                 y_shared=y_shared, h_shared=h_shared, out=out,
+                y_routed_bf16=y_routed_bf16, y_shared_bf16=y_shared_bf16,
                 routed_parts=routed, shared_parts=shared)

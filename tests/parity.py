@@ -16,11 +16,20 @@ SCALE_RTOL, and a row holding an accepted different code is re-evaluated by
 the oracle's down projection on the kernel's codes (as a token whose top-K
 keys tie within the routing margin is evaluated under the kernel's
 selection) before its output is compared.
+
+bf16 expert outputs. The kernel sums each output in FP32 and rounds it to
+bf16 (nearest even); the oracle's value is float64. From the sum of absolute
+products behind it (down_bound), the kernel's FP32 value lies within a bound
+of the oracle's, so its bf16 output must lie between the bf16 roundings of
+the two ends of that interval (assert_bf16_rounding): equal to the oracle's
+rounding except where the oracle's value sits within the bound of a bf16
+midpoint, where either neighbour is valid. h' is then compared with the
+oracle's combine of the kernel's (so validated) bf16 outputs.
 """
 import numpy as np
 
 from oracle import moe as O
-from oracle.e4m3 import decode, encode
+from oracle.e4m3 import decode, encode, round_bf16
 
 RTOL, ATOL_RMS = 8e-3, 1e-3
 SCALE_RTOL = 1e-4        # tile scales fl32(amax / 448): amax accumulated in FP32 vs float64
@@ -94,3 +103,28 @@ def near_tie_rows(hq_gpu, hs_gpu, a32, da, hq_ref, hs_ref, what):
     vo = decode(hq_ref[r, c])
     ratio = np.abs(x - 0.5 * (vg + vo)) / np.maximum(dx, 1e-300)
     return np.unique(r), float(ratio.max())
+
+
+def down_bound(hq, hs, w):
+    """Bound on |y_kernel - y| for the down projection y = H W_down^T of FP8
+    intermediate rows (hq, hs): I/128 K blocks promoted in FP32."""
+    H = np.abs(O.dequant_1x128(hq, hs))
+    kb = H.shape[1] // 128
+    return ROUNDINGS(kb) * EPS32 * (H @ np.abs(O.dequant_128x128(w["down_q"], w["down_s"])).T)
+
+
+def assert_bf16_rounding(gpu, ref, bound, what):
+    """gpu: the kernel's bf16 outputs (as float64); ref: the oracle's float64
+    values; bound: how far the kernel's FP32 sums can be from ref. Each output
+    must be a bf16 rounding of some value within the bound. Returns the number
+    of outputs that took the other side of a bf16 midpoint."""
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    lo, hi, mid = round_bf16(ref - bound), round_bf16(ref + bound), round_bf16(ref)
+    bad = (gpu < lo) | (gpu > hi)
+    if bad.any():
+        i = np.unravel_index(np.argmax(bad), bad.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outputs are no bf16 rounding of the "
+                             f"oracle's value within the accumulation bound; first at {i}: gpu={gpu[i]} "
+                             f"ref={ref[i]} bound={np.broadcast_to(bound, ref.shape)[i]}")
+    return int((gpu != mid).sum())

@@ -16,6 +16,7 @@ import torch.multiprocessing as mp
 import workloads
 from fine_grained_fp8_sigmoid_b200.ep import split_plan
 from oracle import moe as O
+from oracle.e4m3 import round_bf16
 
 
 def _free_port():
@@ -63,7 +64,8 @@ class OracleOps:
                 y[off[g]:off[g + 1]], _ = O.expert_ffn(xq_perm[off[g]:off[g + 1]].numpy(),
                                                        xs_perm[off[g]:off[g + 1]].numpy(), self.w[g])
         ysh, _ = O.expert_ffn(xq.numpy(), xs.numpy(), self.w[self.E])
-        return torch.from_numpy(y), torch.from_numpy(ysh)
+        # the expert outputs leave as bf16 values, as the GPU's do
+        return torch.from_numpy(round_bf16(y)), torch.from_numpy(round_bf16(ysh))
 
     def gather_rows(self, src, idx):
         return src[idx.long()].contiguous()

@@ -15,7 +15,8 @@ from oracle.e4m3 import round_fp32
 
 pytestmark = pytest.mark.gpu
 
-from tests.parity import accumulation_bound, assert_close, f64, near_tie_rows  # noqa: F401
+from tests.parity import (accumulation_bound, assert_bf16_rounding, assert_close, down_bound,  # noqa: F401
+                          f64, near_tie_rows)
 
 
 # ---------------------------------------------------------------- quantisers
@@ -265,12 +266,17 @@ def test_permute_bit_exact(lib, T, N, K, pattern):
 # ---------------------------------------------------------------- combine, bias
 
 @pytest.mark.parametrize("T,K,d", [(1, 1, 8), (333, 2, 256), (1000, 8, 7168)])
-def test_combine(lib, T, K, d):
+@pytest.mark.parametrize("ydt", [torch.bfloat16, torch.float32])
+def test_combine(lib, T, K, d, ydt):
+    """moe_combine on the layer's bf16 expert rows, and moe_combine_fp32 on
+    FP32 rows (the backward's). The kernel's FP32 sum of K + 2 terms is within
+    (K + 2) roundings of 2^-24 |term| of the float64 sum, so h' is at most one
+    bf16 step plus that from the oracle's value."""
     from fine_grained_fp8_sigmoid_b200 import binding as B
     g = torch.Generator().manual_seed(T + d)
     u = torch.randn(T, d, generator=g).to(torch.bfloat16)
-    ysh = torch.randn(T, d, generator=g) * 3.0
-    yp = torch.randn(T * K, d, generator=g) * 3.0
+    ysh = (torch.randn(T, d, generator=g) * 3.0).to(ydt)
+    yp = (torch.randn(T * K, d, generator=g) * 3.0).to(ydt)
     inv = torch.randperm(T * K, generator=g).reshape(T, K).to(torch.int32)
     gt = torch.rand(T, K, generator=g)
     gt = gt / gt.sum(dim=1, keepdim=True)
@@ -280,6 +286,15 @@ def test_combine(lib, T, K, d):
     ref = O.combine(u.double().numpy(), yp.double().numpy(), ysh.double().numpy(),
                     inv.numpy(), gt.double().numpy())
     assert_close(f64(out), ref, "combine")
+    g64, inv_ = gt.double().numpy(), inv.numpy()
+    yp64 = yp.double().numpy()
+    terms = np.abs(u.double().numpy()) + np.abs(ysh.double().numpy())
+    for k in range(K):
+        terms += np.abs(g64[:, k:k + 1] * yp64[inv_[:, k]])
+    step = np.ldexp(1.0, np.frexp(np.abs(ref))[1] - 8)
+    off = np.abs(f64(out) - ref)
+    assert np.all(off <= step + 2 * (K + 2) * 2.0 ** -24 * terms), \
+        "combine: more than one bf16 step plus the FP32 sum's rounding from the float64 sum"
 
 
 @pytest.mark.parametrize("N,T,K", [(8, 64, 2), (256, 8192, 8), (64, 4095, 6), (256, 0, 8)])
@@ -350,8 +365,8 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
     wg, wu, wd = stack("gate_q", torch.uint8), stack("up_q", torch.uint8), stack("down_q", torch.uint8)
     sg, su, sd = stack("gate_s", torch.float32), stack("up_s", torch.float32), stack("down_s", torch.float32)
     off = torch.from_numpy(offsets).cuda()
-    y_perm = torch.empty(Ppad, d, dtype=torch.float32, **dev)
-    y_sh = torch.empty(T, d, dtype=torch.float32, **dev)
+    y_perm = torch.empty(Ppad, d, dtype=torch.bfloat16, **dev)
+    y_sh = torch.empty(T, d, dtype=torch.bfloat16, **dev)
     ws = torch.empty(B.moe_grouped_gemm_fp8_workspace(T, K_r, d, I), dtype=torch.uint8, **dev)
     B.moe_grouped_gemm_fp8(xq_pd, xs_pd, off, cu(xq, torch.uint8), cu(xs, torch.float32),
                            wg, wu, wd, sg, su, sd, y_perm, y_sh, ws)
@@ -377,6 +392,9 @@ def test_grouped_gemm_fp8(lib, d, I, counts, T):
             ref[flip] = O.expert_down(hq_g[g0 + flip], hs_g[g0 + flip], experts[i])
         got = yp[a:b_] if i < N_r else f64(y_sh)
         assert_close(got, ref, f"expert {i}")
+        # bf16 outputs: the rounding of the kernel's FP32 sums (near-ties either way)
+        assert_bf16_rounding(got, ref, down_bound(hq_g[g0:g0 + b_ - a], hs_g[g0:g0 + b_ - a], experts[i]),
+                             f"expert {i} bf16 rounding")
 
 
 @pytest.mark.parametrize("d,I,T,K,N_r", [(512, 256, 300, 3, 7), (2048, 1024, 700, 6, 16),
@@ -407,8 +425,8 @@ def test_grouped_gemm_gather_matches_materialised(lib, d, I, T, K, N_r):
     st_d, off_d = cu(sorted_token, torch.int32), cu(offsets, torch.int32)
     outs = []
     for gathered in (False, True):
-        y_perm = torch.full((P, d), float("nan"), dtype=torch.float32, **dev)
-        y_sh = torch.full((T, d), float("nan"), dtype=torch.float32, **dev)
+        y_perm = torch.full((P, d), float("nan"), dtype=torch.bfloat16, **dev)
+        y_sh = torch.full((T, d), float("nan"), dtype=torch.bfloat16, **dev)
         ws = torch.zeros(B.moe_grouped_gemm_fp8_workspace(T, K, d, I), dtype=torch.uint8, **dev)
         if gathered:
             B.moe_grouped_gemm_fp8_gather(st_d, off_d, xq_d, xs_d, *W, y_perm, y_sh, ws)
@@ -443,6 +461,8 @@ def test_grouped_gemm_gather_matches_materialised(lib, d, I, T, K, N_r):
             ref[flip] = O.expert_down(hq_g[h0 + flip], hs_g[h0 + flip], experts[i])
         got = yp[offsets[i]:offsets[i + 1]] if i < N_r else ysh
         assert_close(got, ref, f"expert {i}")
+        assert_bf16_rounding(got, ref, down_bound(hq_g[h0:h0 + n], hs_g[h0:h0 + n], experts[i]),
+                             f"expert {i} bf16 rounding")
 
 
 # ---------------------------------------------------------------- failure path

@@ -19,7 +19,7 @@ import torch
 
 import workloads
 from oracle import moe as O
-from tests.parity import accumulation_bound, assert_close, f64, near_tie_rows
+from tests.parity import accumulation_bound, assert_bf16_rounding, assert_close, down_bound, f64, near_tie_rows
 from tests.test_gpu_kernels import _check_routing
 
 pytestmark = pytest.mark.gpu
@@ -155,11 +155,26 @@ def _run(cfg, weights_on, all_tokens=False):
     print(f"[parity] {cfg.name} T={cfg.T}: {flip.size} of {hq_g.shape[0]} intermediate rows hold a "
           f"near-tie code (max distance to the boundary {dist:.3g} of the bound)")
 
-    assert_close(f64(layer.y_shared)[sample], y_s, "shared expert")
+    # bf16 expert outputs: each the rounding of the kernel's FP32 sum, which
+    # lies within the accumulation bound of the oracle's value (near a bf16
+    # midpoint either neighbour is valid); h' is then checked against the
+    # oracle's combine of those outputs
+    yb_s = f64(layer.y_shared)[sample]
     yp = f64(layer.y_perm)
+    yb_r = np.concatenate([yp[inv[t]] for t in sample])
+    assert_close(yb_s, y_s, "shared expert")
     for j, t in enumerate(sample):
-        assert_close(yp[inv[t]], y_r[j * K:(j + 1) * K], f"routed rows of token {t}")
-    out_ref = O.combine(un[sample], y_r, y_s, np.arange(S * K).reshape(S, K), ref["gates"][sample])
+        assert_close(yb_r[j * K:(j + 1) * K], y_r[j * K:(j + 1) * K], f"routed rows of token {t}")
+    yb = np.concatenate([yb_r, yb_s])
+    y64 = np.concatenate([y_r, y_s])
+    n_flip = 0
+    for s_ in np.unique(slot_of):
+        rr = np.nonzero(slot_of == s_)[0]
+        n_flip += assert_bf16_rounding(yb[rr], y64[rr], down_bound(hq_g[rr], hs_g[rr], quant[int(s_)]),
+                                       f"{cfg.name} expert {int(s_)} outputs")
+    print(f"[parity] {cfg.name} T={cfg.T}: {n_flip} of {yb.size} bf16 expert outputs on the other side "
+          f"of a rounding midpoint (within the accumulation bound)")
+    out_ref = O.combine(un[sample], yb_r, yb_s, np.arange(S * K).reshape(S, K), ref["gates"][sample])
     assert_close(f64(out)[sample], out_ref, "h'")
     return layer
 

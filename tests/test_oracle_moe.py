@@ -355,15 +355,18 @@ def test_all_experts_selected_equals_dense_gated_sum():
     zero = _const_expert(256, 128, 0, 0, 0)
     get = lambda s: zero if s == cfg.N_r else prov(s)
     r = moe.moe_forward(u, e, b, cfg.K_r, get)
-    # dense: every expert on every token, gate s_i / sum_j s_j
+    # dense: every expert on every token, gate s_i / sum_j s_j, each expert's
+    # output taken as bf16 (the layer's expert-output type)
     s = moe.router_scores(u, e)
     xq, xs = moe.quant_1x128(u)
     acc = u.copy()
     for i in range(4):
         y, _ = moe.expert_ffn(xq, xs, prov(i))
-        acc += (s[:, i] / s.sum(axis=1))[:, None] * y
-    assert np.allclose(r["out"], round_bf16(acc), rtol=2 ** -8, atol=0)
-    assert np.abs(r["out"] - round_bf16(acc)).max() <= 2 ** -8 * np.abs(acc).max()
+        acc += (s[:, i] / s.sum(axis=1))[:, None] * round_bf16(y)
+    # equal bit for bit (the float64 sums differ only in order, far below a
+    # bf16 step); unrounded expert outputs would move a few dozen of these
+    # 5120 outputs by one bf16 step
+    assert np.array_equal(r["out"], round_bf16(acc))
 
 
 def test_token_sample_matches_full_forward():

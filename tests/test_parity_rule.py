@@ -66,3 +66,23 @@ def test_accumulation_bound_grows_with_the_absolute_sums():
     assert np.all(da > 0) and np.all(da[1] > 2 * da[0])
     zero = accumulation_bound(xq, xs, w, np.zeros((2, I)), np.zeros((2, I)))
     assert np.all(zero == 0.0)
+
+
+def test_bf16_output_rule():
+    from oracle.e4m3 import round_bf16
+    from tests.parity import assert_bf16_rounding
+    rng = np.random.default_rng(3)
+    ref = rng.standard_normal(1000)
+    # the correctly rounded outputs pass with any bound, and count no flips
+    assert assert_bf16_rounding(round_bf16(ref), ref, 0.0, "exact") == 0
+    # one bf16 step off is rejected when the bound is far below a step
+    step = np.ldexp(1.0, np.frexp(np.abs(ref))[1] - 8)
+    with pytest.raises(AssertionError):
+        assert_bf16_rounding(round_bf16(ref) + step, ref, 1e-12, "one step off")
+    # a value just above a bf16 midpoint may come out on either side when the
+    # bound reaches the midpoint, and not when it does not
+    mid = 1.0 + 2.0 ** -8                       # between 1 and 1 + 2^-7
+    v = np.array([mid + 2.0 ** -30])
+    assert assert_bf16_rounding(np.array([1.0]), v, 2.0 ** -29, "near tie") == 1
+    with pytest.raises(AssertionError):
+        assert_bf16_rounding(np.array([1.0]), v, 2.0 ** -31, "outside the bound")
