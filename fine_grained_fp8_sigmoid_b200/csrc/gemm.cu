@@ -44,9 +44,11 @@
 //            Epilogue: SwiGLU a = silu(G) * U, 1x128 requantisation to E4M3
 //            (the tile is exactly one 128-channel scale tile), written to H.
 //   phase 2: per tile (group g, 128 rows, 256 output channels):
-//            A = H, B = W_down rows; the FP32 accumulators leave through
-//            shared memory and TMA stores (the combine adds them to the
-//            residual and rounds once).
+//            A = H, B = W_down rows; the FP32 accumulators are rounded to
+//            bf16 and leave through shared memory and TMA stores (the
+//            combine adds them to the residual in FP32). The backward's
+//            GEMMs run this phase on its own with FP32 outputs, and in a
+//            K-grouped mode where every group has its own K range.
 // Tiles are numbered group-major (shared expert last), then row tile, then
 // column tile. The first wave is dealt by block index; after it each CTA
 // claims the next number from a counter in the workspace, so the tiles in
