@@ -111,9 +111,10 @@ __device__ __forceinline__ void topk_store(const int (&ii)[KMAX], const float (&
   }
 }
 
-// sigmoid with the hardware exponential and reciprocal (relative error
-// ~1e-6, far inside the routing acceptance margin); sigmoid(0) = 0.5 exactly
-__device__ __forceinline__ float sigmoid_fast(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+// sigmoid with the hardware exponential and approximate division (relative
+// error ~1e-6, far inside the routing acceptance margin); sigmoid(0) = 0.5
+// exactly, and the limits 0 (z -> -inf: 1 / inf) and 1 hold
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 
 // top-K of (key, index) pairs, keys descending; strict comparison, so an
 // equal key inserted later (a higher index) stays behind

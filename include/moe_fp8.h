@@ -118,7 +118,7 @@ MOE_API int moe_quant_128x128(const float* w, int rows, int cols, uint8_t* q,
  *              descending, equal keys by lower index first
  *   gates      [T][K_r] FP32: g = s_sel / sum(s_sel), in the same order
  * The logits u . e run on the tensor cores in BF16 with FP32 accumulation; the
- * affinity uses the hardware exponential and reciprocal (relative error
+ * affinity uses the hardware exponential and approximate division (relative error
  * ~1e-6); the key s + b is formed in FP32. With few 128-token tiles the launch
  * is a set of thread-block clusters (2..8 CTAs per tile) that split d and add
  * their partial logits in a fixed order, so results do not depend on the
