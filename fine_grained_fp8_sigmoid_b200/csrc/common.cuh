@@ -91,16 +91,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// Warp-uniform wait: lane 0 polls, the outcome is broadcast, so the whole
-// warp either proceeds (and may then issue .sync.aligned tcgen05 ops) or
-// gives up together.
+// Warp-uniform wait: every lane polls and one vote combines the outcomes,
+// so the whole warp either proceeds (and may then issue .sync.aligned
+// tcgen05 ops) or gives up together.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = kWaitLimitNs) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, limit_ns) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
-  return ok != 0;
+  const bool ok = mbar_wait(bar, parity, abort, limit_ns);
+  return __all_sync(0xffffffffu, ok);
 }
 
 // ---------------------------------------------------------------- TMA
