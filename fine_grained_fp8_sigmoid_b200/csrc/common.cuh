@@ -278,6 +278,13 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// One wait for two register sets loaded by tmem_ld32_async.
+__device__ __forceinline__ void tmem_wait_ld2(uint32_t (&a)[32], uint32_t (&b)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(a[i]), "+r"(b[i]));
+}
+
 // Register budget changes for warp-specialised kernels (all threads of a
 // warpgroup execute them together). The values used with a launch of T
 // threads at R registers must satisfy: sum over warpgroups of 128 * regs <=

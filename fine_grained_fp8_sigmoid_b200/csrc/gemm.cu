@@ -664,14 +664,16 @@ __global__ void __launch_bounds__(THREADS, 1)
           // the operands usually land well before the partial buffer is free:
           // check them first, so that only the buffer's wait sits between the
           // epilogue's release and the next MMAs
+          // descriptors first: only the waits sit between the epilogue's
+          // release and the MMAs
+          const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
+          const uint64_t ad = sw128_kmajor_desc(a_addr);
+          const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
+          const uint32_t d_tmem = tmem + buf * BN;
           if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
           if (!mbar_wait(&sm.tempty[buf], tphase ^ 1, abort)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
-          const uint64_t ad = sw128_kmajor_desc(a_addr);
-          const uint32_t d_tmem = tmem + buf * BN;
           if (!tl.narrow) {
-            const uint64_t bd = sw128_kmajor_desc(a_addr + A_BYTES);
 #pragma unroll
             for (int k = 0; k < BK / 32; ++k) umma_f8f6f4(d_tmem, ad + 2 * k, bd + 2 * k, idesc, k > 0);
           } else {
@@ -790,16 +792,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t ra[32], rb[32];
         tmem_ld32_async(ta + c0, ra);
         tmem_ld32_async(ta + c0 + 32, rb);
-        tmem_wait_ld(ra);
-        tmem_wait_ld(rb);
+        tmem_wait_ld2(ra, rb);
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[j] = fmaf(f01, __uint_as_float(ra[j]), acc[j]);
         tmem_ld32_async(ta + c2, ra);
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[32 + j] = fmaf(f01, __uint_as_float(rb[j]), acc[32 + j]);
         tmem_ld32_async(ta + c2 + 32, rb);
-        tmem_wait_ld(ra);
-        tmem_wait_ld(rb);
+        tmem_wait_ld2(ra, rb);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.tempty[buf]);
