@@ -57,3 +57,23 @@ def test_clock_samples_inside_the_region_only():
     assert s["samples"] == 3 and s["sm_mhz"] == 1700 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"]
     assert bench.ClockSampler.parse([], t0, t0 + 1)["reasons"] == ["unsampled"]
+
+
+def test_gemm_traffic_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
+    """The bench reports a committed DRAM-traffic figure only while the GEMM
+    source hashes to the value recorded beside it."""
+    import shutil
+    cfg = workloads.CONFIGS["prefill"]
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    csrc = root / "fine_grained_fp8_sigmoid_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    shutil.copy(bench.os.path.join(bench.ROOT, "fine_grained_fp8_sigmoid_b200", "csrc", "gemm.cu"), csrc / "gemm.cu")
+    sha = bench.gemm_source_sha256(str(csrc))
+    prof = root / "profiles" / "grouped_gemm_prefill_traffic.md"
+    prof.write_text(f"gemm_cu_sha256: {sha}\ndram_bytes_per_call: 123456789\n")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.gemm_traffic(cfg) == 123456789.0
+    (csrc / "gemm.cu").write_text((csrc / "gemm.cu").read_text() + "// changed\n")
+    assert bench.gemm_traffic(cfg) is None
+    assert bench.gemm_traffic(workloads.CONFIGS["decode"]) is None     # no profile for it

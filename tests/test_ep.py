@@ -115,6 +115,19 @@ def test_split_plan():
     assert off.tolist() == [0, 2, 2, 3, 3, 6, 9]
 
 
+def test_split_plan_with_idle_ranks_and_experts():
+    # 4 ranks, 2 experts each; this rank routes nothing to ranks 1 and 3, and
+    # receives nothing at all from rank 2
+    counts = np.array([5, 0, 0, 0, 1, 2, 0, 0])
+    recv = np.array([[3, 0], [0, 0], [0, 0], [1, 7]])
+    send, rv, off = split_plan(counts, recv, 4, 2)
+    assert send == [5, 0, 3, 0] and rv == [3, 0, 0, 8]
+    assert off.tolist() == [0, 3, 3, 3, 3, 3, 3, 4, 11]
+    # nothing anywhere: all splits zero, offsets all zero
+    send, rv, off = split_plan(np.zeros(8, np.int64), np.zeros((4, 2), np.int64), 4, 2)
+    assert send == [0] * 4 and rv == [0] * 4 and off.tolist() == [0] * 9
+
+
 @pytest.mark.parametrize("world", [2, 4])
 def test_ep_ranks_match_single_rank_oracle(world):
     ctx = mp.get_context("spawn")
