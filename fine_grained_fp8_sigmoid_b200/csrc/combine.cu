@@ -217,6 +217,6 @@ extern "C" const char* moe_status_string(int status) {
   }
 }
 
-extern "C" int moe_version(void) { return 100; }
+extern "C" int moe_version(void) { return 200; }
 
 extern "C" const char* moe_last_error_detail(void) { return moe::last_error_buf(); }

@@ -62,7 +62,10 @@ typedef enum {
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(int status);
 
-/* Library version, e.g. 100 for 0.1.0. */
+/* Library version, e.g. 200 for 0.2.0. 0.2.0: expert outputs (y_perm,
+ * y_shared of moe_grouped_gemm_fp8 and its variants, the rows moe_combine
+ * reads) are bf16; moe_combine_fp32, moe_kgrouped_gemm_fp8 and
+ * moe_route_quant added; the transposed quantisers write [cols][Ktot]. */
 MOE_API int moe_version(void);
 
 /*

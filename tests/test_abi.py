@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     assert _lib.status_string(0) == "MOE_OK"
     assert _lib.status_string(4) == "MOE_ERR_TIMEOUT"
-    assert lib.moe_version() == 100
+    assert lib.moe_version() == 200
 
 
 def test_workspace_sizes(lib):
