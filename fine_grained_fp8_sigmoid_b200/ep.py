@@ -1,6 +1,7 @@
 """Expert parallelism across the GPUs of one node: the DeepSeekMoE FP8 layer
-with its routed experts sharded over G ranks ("[논문 리뷰] DeepSeek-V3
-Technical Report" review, "학습 인프라 & 최적화": the model trains with EP64;
+with its routed experts sharded over G ranks ("DeepSeek 알고 아는 척 좀
+해보자 – 단편: 671B 파라미터의 괴물, DeepSeek-V3", "학습 인프라 & 최적화": the
+model trains with 64-way expert parallelism;
 "DeepSeek-V3 Teknik Raporu", "Problem ve motivasyon" item 2: the all-to-all
 exchange behind it is a bottleneck).
 

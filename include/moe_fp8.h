@@ -282,8 +282,9 @@ MOE_API int moe_grouped_gemm_fp8_gather(const int32_t* sorted_token,
  * P = T * K_r; the shared expert runs on T rows of xq (slot N_groups). Used
  * where the routed rows are not this batch's T * K_r pairs: under expert
  * parallelism a GPU runs its local experts on the rows the other GPUs sent
- * it ("[논문 리뷰] DeepSeek-V3 Technical Report" review, "학습 인프라 &
- * 최적화": EP64). Same products, scales, layouts and limits as
+ * it ("DeepSeek 알고 아는 척 좀 해보자 – 단편: 671B 파라미터의 괴물,
+ * DeepSeek-V3", "학습 인프라 & 최적화": 64-way expert parallelism). Same
+ * products, scales, layouts and limits as
  * moe_grouped_gemm_fp8 (weights stacked over N_groups + 1 slots); P may be 0
  * (then xq_perm, xs_perm and y_perm may be NULL); T must be >= 1.
  */
