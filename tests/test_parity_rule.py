@@ -86,3 +86,15 @@ def test_bf16_output_rule():
     assert assert_bf16_rounding(np.array([1.0]), v, 2.0 ** -29, "near tie") == 1
     with pytest.raises(AssertionError):
         assert_bf16_rounding(np.array([1.0]), v, 2.0 ** -31, "outside the bound")
+
+
+def test_bf16_output_rule_rejects_truncation():
+    # a kernel that truncated its FP32 sums to bf16 instead of rounding to
+    # nearest even is caught, even with a generous accumulation bound
+    from tests.parity import assert_bf16_rounding
+    rng = np.random.default_rng(4)
+    ref = rng.standard_normal(4096)
+    bits = ref.astype(np.float32).view(np.uint32) & np.uint32(0xFFFF0000)
+    truncated = bits.view(np.float32).astype(np.float64)
+    with pytest.raises(AssertionError):
+        assert_bf16_rounding(truncated, ref, 1e-9 * np.abs(ref), "truncated")
